@@ -1,0 +1,401 @@
+"""Benchmark of the W4A4 + low-rank linear layer on B200.
+
+One step = one pass of the whole hot path (kernel 1: smoothing + NVFP4 activation quantization +
+low-rank down-projection; kernel 2: block-scaled FP4 GEMM + up-projection + epilogue) over every
+linear of the workload, on seeded synthetic inputs already resident in HBM. L2 is flushed (a 256 MB
+write) between timed steps, outside the timed events. Timing: CUDA events on the launching stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl svdq|reference]
+
+N > 1 runs under torchrun as independent replicas (the layer has no exchange step), weak scaling.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_diffusion_transformer_svdquant_b200 import synth  # noqa: E402
+
+METRIC = "W4A4+low-rank linear TFLOPS, % of B200 dense FP4 peak; tokens/s per layer"
+DEFAULT_WORKLOAD = "qkv_2048"
+FP4_PER_BF16 = 4.0   # nominal dense FP4 / dense bf16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+FLUSH_BYTES = 256 << 20
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs (read-only)."""
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period, self.samples, self.reasons = index, period_s, [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: clocks are reported as unavailable
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {"hw_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+                 "hw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+                 "sw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+                 "sw_power_cap": getattr(nv, "nvmlClocksThrottleReasonSwPowerCap", 0x4)}
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for k, bit in names.items():
+                    if mask & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def layer_flops(spec):
+    return 2.0 * spec.M * spec.N * spec.K, 2.0 * spec.M * spec.r * (spec.K + spec.N)
+
+
+def kernel1_bytes(spec):
+    """Algorithmic HBM bytes of kernel 1: read X (bf16), write codes + scales + U (bf16)."""
+    return spec.M * spec.K * 2 + spec.M * spec.K // 2 + spec.M * spec.K // 16 + spec.M * spec.r * 2
+
+
+# ---------------------------------------------------------------------------------------------- GPU arm
+def build_layers(wl, dev):
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+    from bit_diffusion_transformer_svdquant_b200.prepare import prepare_layer
+
+    layers = []
+    prev_out = None
+    for spec in wl.layers:
+        d = synth.make_linear_inputs(spec)
+        chained = wl.name.startswith("mlp") and prev_out is not None
+        X = prev_out if chained else d["X"].to(dev)
+        p = prepare_layer(X, d["W"].to(dev), spec.r, dev)
+        w = svdq.PackedWeight(p["R"], p["L1s"], p["L2"], p["inv_lambda"], swiglu=spec.swiglu)
+        del p
+        g_x = svdq.calibrate_act(X, w)
+        act = svdq.QuantizedAct(spec.M, spec.K, spec.r, dev)
+        bias = d["bias"].to(dev) if spec.bias else None
+        n_out = spec.N // 2 if spec.swiglu else spec.N
+        Y = torch.empty(spec.M, n_out, dtype=torch.bfloat16, device=dev)
+        layers.append({"spec": spec, "X": X, "w": w, "g_x": g_x, "act": act, "bias": bias, "Y": Y})
+        if wl.name.startswith("mlp"):
+            svdq.quantize_act(X, w, g_x, act)
+            svdq.gemm(act, w, bias, out=Y)
+            prev_out = Y
+    torch.cuda.synchronize(dev)
+    return layers
+
+
+def run_step(layers, ev=None):
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+    for i, L in enumerate(layers):
+        svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
+        if ev is not None:
+            ev[i].record()
+        svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
+
+
+def gpu_arm(args, rank, world, dev):
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+
+    wl = synth.WORKLOADS[args.workload]
+    layers = build_layers(wl, dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        run_step(layers)
+    torch.cuda.synchronize(dev)
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out during warm-up")
+
+    K = args.steps
+    n_l = len(layers)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    mids = [[torch.cuda.Event(enable_timing=True) for _ in range(n_l)] for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    # kernel-level events: quantize (kernel 1) and GEMM (kernel 2) of every layer
+    k_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+              torch.cuda.Event(enable_timing=True)) for _ in range(n_l)] for _ in range(K)]
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_wall = time.perf_counter()
+        for s in range(K):
+            flush.zero_()
+            starts[s].record(stream)
+            for i, L in enumerate(layers):
+                e0, e1, e2 = k_ev[s][i]
+                e0.record(stream)
+                svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
+                e1.record(stream)
+                svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
+                e2.record(stream)
+            ends[s].record(stream)
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out during the timed region")
+
+    step_ms = [starts[s].elapsed_time(ends[s]) for s in range(K)]
+    total_ms = float(sum(step_ms))
+    k1_ms = [[k_ev[s][i][0].elapsed_time(k_ev[s][i][1]) for s in range(K)] for i in range(n_l)]
+    k2_ms = [[k_ev[s][i][1].elapsed_time(k_ev[s][i][2]) for s in range(K)] for i in range(n_l)]
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    flops_main = sum(layer_flops(L["spec"])[0] for L in layers)
+    flops_lr = sum(layer_flops(L["spec"])[1] for L in layers)
+    tokens = layers[0]["spec"].M
+    ms_per_step = total_ms / K
+    value = world * flops_main / (ms_per_step * 1e-3) / 1e12
+
+    # dominant kernel: the GEMM of the largest layer
+    big = max(range(n_l), key=lambda i: layer_flops(layers[i]["spec"])[0])
+    spec_b = layers[big]["spec"]
+    k2_avg = statistics.mean(k2_ms[big])
+    peaks = read_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    gemm_flops = sum(layer_flops(spec_b))
+    achieved = gemm_flops / (k2_avg * 1e-3) / 1e12
+    k1_avg = [statistics.mean(k1_ms[i]) for i in range(n_l)]
+    k1_gbs = [kernel1_bytes(layers[i]["spec"]) / (k1_avg[i] * 1e-3) / 1e9 for i in range(n_l)]
+
+    e2e = e2e_arm(args, layers, dev, world)
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) + bf16 low-rank, fp32 acc",
+        "data": "synthetic (seeded; FLUX-class token counts)",
+        "config": {"workload": wl.name, "description": wl.description,
+                   "layers": [f"{L['spec'].M}x{L['spec'].K}x{L['spec'].N} r={L['spec'].r}"
+                              + (" swiglu" if L["spec"].swiglu else "") + (" bias" if L["spec"].bias else "")
+                              for L in layers],
+                   "l2": "flushed between timed steps (256 MB write, outside the events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "tokens_per_s": round(world * tokens / (ms_per_step * 1e-3), 1),
+        "tflops_incl_lowrank": round(world * (flops_main + flops_lr) / (ms_per_step * 1e-3) / 1e12, 2),
+        "frac_fp4_peak_e2e": round(value / world / fp4_peak, 4),
+        "kernels": {
+            "quantize_act_us": [round(x * 1e3, 2) for x in k1_avg],
+            "quantize_act_gbs": [round(x, 1) for x in k1_gbs],
+            "quantize_act_frac_hbm": [round(x / peaks["hbm_gbs"], 4) for x in k1_gbs],
+            "gemm_us": [round(statistics.mean(k2_ms[i]) * 1e3, 2) for i in range(n_l)],
+        },
+        "roofline": {"bound": "tensor", "kernel": "svdq_gemm_kernel", "achieved": round(achieved, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
+                     "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_PER_BF16}"
+                                    " (nominal dense FP4/bf16 ratio)",
+                     "algorithmic": f"{gemm_flops / 1e9:.1f} GFLOP per launch (2MNK + 2MrN)"},
+        "e2e": e2e,
+        "gpu_launches": 2 * n_l * K,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": round(t_wall, 3),
+    }
+    return out
+
+
+def e2e_arm(args, layers, dev, world):
+    """The same metric through the public API with host buffers: every step copies the first layer's
+    X from pinned host memory, runs the layer(s), and copies the last output back to pinned host."""
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+    stream = torch.cuda.current_stream(dev)
+    X_host = layers[0]["X"].cpu().pin_memory()
+    Y_last = layers[-1]["Y"]
+    Y_host = torch.empty(Y_last.shape, dtype=Y_last.dtype).pin_memory()
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        layers[0]["X"].copy_(X_host, non_blocking=True)
+        run_step(layers)
+        Y_host.copy_(Y_last, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        layers[0]["X"].copy_(X_host, non_blocking=True)
+        run_step(layers)
+        Y_host.copy_(Y_last, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out in the end-to-end loop")
+    flops = sum(layer_flops(L["spec"])[0] for L in layers)
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": X_host.numel() * X_host.element_size(),
+            "d2h_bytes_per_step": Y_host.numel() * Y_host.element_size()}
+
+
+# ---------------------------------------------------------------------------------------------- CPU oracle
+def oracle_setup(wl, rows_hint=64):
+    """The oracle's offline preparation for every layer of the workload (not timed)."""
+    from oracle import svdquant
+    prepared = []
+    for spec in wl.layers:
+        d = synth.make_linear_inputs(spec)
+        X, W = synth.bf16_values(d["X"]), synth.bf16_values(d["W"])
+        p = svdquant.prepare_layer(X, W, spec.r)
+        g_x = svdquant.calibrate_activation_scale(X, p["inv_lambda"])
+        wq = svdquant.quantize_weight(p["R"])
+        b = synth.bf16_values(d["bias"]) if spec.bias else None
+        prepared.append({"spec": spec, "X": X, "p": p, "g_x": g_x, "wq": wq, "b": b})
+    return prepared
+
+
+def oracle_step(prepared, rows):
+    from oracle import svdquant
+    for P in prepared:
+        svdquant.layer_forward(P["X"][:rows], P["p"], P["g_x"], P["wq"], P["b"], P["spec"].swiglu)
+
+
+def choose_rows(prepared, target_s):
+    rows = 64
+    t0 = time.perf_counter()
+    oracle_step(prepared, rows)
+    dt = time.perf_counter() - t0
+    M = prepared[0]["spec"].M
+    return int(max(16, min(M, rows * target_s / max(dt, 1e-3))))
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"), default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(wl, target_s=15.0):
+    prepared = oracle_setup(wl)
+    rows = choose_rows(prepared, target_s)
+    t0 = time.perf_counter()
+    oracle_step(prepared, rows)
+    dt = time.perf_counter() - t0
+    flops = sum(2.0 * rows * P["spec"].N * P["spec"].K for P in prepared)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{rows} of {prepared[0]['spec'].M} token rows through every layer of {wl.name} "
+                      f"(fp64 numpy oracle, weights prepared offline), {dt:.1f} s"}
+
+
+def reference_arm(args):
+    wl = synth.WORKLOADS[args.workload]
+    prepared = oracle_setup(wl)
+    rows = choose_rows(prepared, target_s=min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_step(prepared, rows)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(prepared, rows)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    flops = sum(2.0 * rows * P["spec"].N * P["spec"].K for P in prepared)
+    value = flops / (ms * 1e-3) / 1e12
+    sample = (f"{rows} of {prepared[0]['spec'].M} token rows per step through every layer of {wl.name} "
+              f"(fp64 numpy oracle on host cores)")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": wl.name, "description": wl.description},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args)), flush=True)
+        return
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    try:
+        out = gpu_arm(args, rank, world, dev)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,249 @@
+"""ctypes binding of libsvdq.so (include/svdq.h). Argument marshalling only: every step of the layer
+runs in the library's CUDA kernels; torch provides device memory and the current stream.
+
+There is no fallback: if the library is missing or the device is not sm_100a, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from ctypes import POINTER, byref, c_char_p, c_int, c_size_t, c_ulonglong, c_void_p
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsvdq.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "svdq.h")
+
+EPI_NONE, EPI_BIAS, EPI_SWIGLU, EPI_BIAS_SWIGLU = 0, 1, 2, 3
+OUT_BF16, OUT_F32 = 0, 1
+STATUS_NAMES = {0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED", 3: "SVDQ_ERR_CUDA",
+                4: "SVDQ_ERR_TIMEOUT"}
+
+
+class SvdqWeight(ctypes.Structure):
+    _fields_ = [("N", c_int), ("K", c_int), ("r", c_int), ("swiglu_interleaved", c_int), ("n_tile", c_int),
+                ("reserved0", c_int), ("codes", c_void_p), ("scales", c_void_p), ("g_w", c_void_p),
+                ("inv_lambda", c_void_p), ("L1s_t", c_void_p), ("L2_t", c_void_p), ("tmap", c_ulonglong * 32)]
+
+
+class SvdqAct(ctypes.Structure):
+    _fields_ = [("M", c_int), ("K", c_int), ("r", c_int), ("M_pad", c_int), ("codes", c_void_p),
+                ("scales", c_void_p), ("U", c_void_p), ("alpha", c_void_p)]
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, func: str, status: int, message: str):
+        super().__init__(f"{func}: {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def _declare(lib):
+    W, A = POINTER(SvdqWeight), POINTER(SvdqAct)
+    sig = {
+        "svdq_weight_bytes": (c_size_t, [c_int, c_int, c_int]),
+        "svdq_act_bytes": (c_size_t, [c_int, c_int, c_int]),
+        "svdq_pack_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,
+                                     c_size_t, W, c_void_p]),
+        "svdq_act_bind": (c_int, [c_int, c_int, c_int, c_void_p, c_size_t, A]),
+        "svdq_calibrate_act": (c_int, [c_void_p, c_int, W, c_void_p, c_void_p]),
+        "svdq_quantize_act": (c_int, [c_void_p, W, c_void_p, A, c_void_p]),
+        "svdq_gemm": (c_int, [A, W, c_void_p, c_int, c_void_p, c_int, c_void_p]),
+        "svdq_export_weight": (c_int, [W, c_void_p, c_void_p, c_void_p]),
+        "svdq_export_act": (c_int, [A, c_void_p, c_void_p, c_void_p]),
+        "svdq_device_status": (c_int, [c_int]),
+        "svdq_watchdog_selftest": (c_int, [c_ulonglong, c_void_p]),
+        "svdq_set_wait_limit_ns": (c_int, [c_ulonglong]),
+        "svdq_status_str": (c_char_p, [c_int]),
+        "svdq_last_error": (c_char_p, []),
+        "svdq_abi_version": (c_int, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+
+
+def lib():
+    """The loaded library. Raises if libsvdq.so has not been built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; "
+                               "g.build()'` (nvcc, sm_100a)")
+        l = ctypes.CDLL(LIB_PATH)
+        _declare(l)
+        _lib = l
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the entry points include/svdq.h declares."""
+    with open(HEADER) as f:
+        return sorted(set(re.findall(r"^SVDQ_API\s+[\w\s\*]+?\b(svdq_\w+)\s*\(", f.read(), re.M)))
+
+
+def _check(func: str, status: int):
+    if status != 0:
+        raise SvdqError(func, status, lib().svdq_last_error().decode())
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, ndim=None):
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {t.dtype} on {t.device}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got {tuple(t.shape)}")
+
+
+class PackedWeight:
+    """One layer's packed weight (device buffer + svdq_weight descriptor)."""
+
+    def __init__(self, R: torch.Tensor, L1s: torch.Tensor | None, L2: torch.Tensor | None,
+                 inv_lambda: torch.Tensor, swiglu: bool = False):
+        _need(R, torch.float32, "R", 2)
+        _need(inv_lambda, torch.float32, "inv_lambda", 1)
+        N, K = R.shape
+        r = 0 if L1s is None else L1s.shape[1]
+        if r:
+            _need(L1s, torch.bfloat16, "L1s", 2)
+            _need(L2, torch.bfloat16, "L2", 2)
+            if tuple(L1s.shape) != (K, r) or tuple(L2.shape) != (r, N):
+                raise ValueError("L1s must be [K, r] and L2 [r, N]")
+        nbytes = lib().svdq_weight_bytes(N, K, r)
+        if nbytes == 0:
+            raise SvdqError("svdq_weight_bytes", 2, f"unsupported shape N={N} K={K} r={r}")
+        self.device = R.device
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=R.device)
+        self.desc = SvdqWeight()
+        with torch.cuda.device(R.device):
+            _check("svdq_pack_weight", lib().svdq_pack_weight(
+                _ptr(R), _ptr(L1s) if r else None, _ptr(L2) if r else None, _ptr(inv_lambda), N, K, r,
+                1 if swiglu else 0, _ptr(self.buf), nbytes, byref(self.desc), _stream(R.device)))
+        self.N, self.K, self.r, self.swiglu = N, K, r, swiglu
+
+    @property
+    def n_tile(self) -> int:
+        return self.desc.n_tile
+
+    def g_w(self) -> torch.Tensor:
+        off = self.desc.g_w - self.buf.data_ptr()
+        return self.buf[off:off + 4].view(torch.float32)
+
+
+class QuantizedAct:
+    """A quantized activation buffer for M rows (codes, scales, U, alpha)."""
+
+    def __init__(self, M: int, K: int, r: int, device):
+        nbytes = lib().svdq_act_bytes(M, K, r)
+        if nbytes == 0:
+            raise SvdqError("svdq_act_bytes", 2, f"unsupported shape M={M} K={K} r={r}")
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.desc = SvdqAct()
+        _check("svdq_act_bind", lib().svdq_act_bind(M, K, r, _ptr(self.buf), nbytes, byref(self.desc)))
+        self.M, self.K, self.r, self.device = M, K, r, self.buf.device
+
+    def _view(self, ptr, nbytes):
+        off = ptr - self.buf.data_ptr()
+        return self.buf[off:off + nbytes]
+
+    def U(self) -> torch.Tensor:
+        return self._view(self.desc.U, self.desc.M_pad * self.r * 2).view(torch.bfloat16).view(self.desc.M_pad, self.r)
+
+    def alpha(self) -> torch.Tensor:
+        return self._view(self.desc.alpha, 4).view(torch.float32)
+
+
+def calibrate_act(X: torch.Tensor, w: PackedWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Static activation scale g_x (device fp32 [1]) from calibration data X [M, K] bf16."""
+    _need(X, torch.bfloat16, "X", 2)
+    out = torch.empty(1, dtype=torch.float32, device=X.device) if out is None else out
+    with torch.cuda.device(X.device):
+        _check("svdq_calibrate_act", lib().svdq_calibrate_act(_ptr(X), X.shape[0], byref(w.desc), _ptr(out),
+                                                              _stream(X.device)))
+    return out
+
+
+def quantize_act(X: torch.Tensor, w: PackedWeight, g_x: torch.Tensor, act: QuantizedAct) -> QuantizedAct:
+    """Kernel 1: smoothing + NVFP4 quantization + low-rank down-projection."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(g_x, torch.float32, "g_x")
+    if X.shape[0] != act.M or X.shape[1] != w.K:
+        raise ValueError("X shape does not match the act buffer / weight")
+    with torch.cuda.device(X.device):
+        _check("svdq_quantize_act", lib().svdq_quantize_act(_ptr(X), byref(w.desc), _ptr(g_x), byref(act.desc),
+                                                            _stream(X.device)))
+    return act
+
+
+def gemm(act: QuantizedAct, w: PackedWeight, bias: torch.Tensor | None = None, epilogue: int | None = None,
+         out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Kernel 2: NVFP4 GEMM + low-rank up-projection + bias / SwiGLU epilogue."""
+    if epilogue is None:
+        epilogue = (EPI_BIAS if bias is not None else EPI_NONE) | (EPI_SWIGLU if w.swiglu else 0)
+    n_out = w.N // 2 if epilogue & EPI_SWIGLU else w.N
+    if out is None:
+        out = torch.empty(act.M, n_out, dtype=out_dtype, device=act.device)
+    _need(out, out_dtype, "out", 2)
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+    code = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
+    with torch.cuda.device(act.device):
+        _check("svdq_gemm", lib().svdq_gemm(byref(act.desc), byref(w.desc), _ptr(bias), epilogue, _ptr(out), code,
+                                            _stream(act.device)))
+    return out
+
+
+def linear(X, w, g_x, bias=None, act=None, out=None, out_dtype=torch.bfloat16):
+    """The whole layer: kernel 1 then kernel 2 on the current stream."""
+    act = QuantizedAct(X.shape[0], w.K, w.r, X.device) if act is None else act
+    quantize_act(X, w, g_x, act)
+    return gemm(act, w, bias, out=out, out_dtype=out_dtype)
+
+
+def export_weight(w: PackedWeight):
+    codes = torch.empty(w.N, w.K // 2, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(w.N, w.K // 16, dtype=torch.uint8, device=w.device)
+    with torch.cuda.device(w.device):
+        _check("svdq_export_weight", lib().svdq_export_weight(byref(w.desc), _ptr(codes), _ptr(scales),
+                                                              _stream(w.device)))
+    return codes, scales
+
+
+def export_act(act: QuantizedAct):
+    codes = torch.empty(act.M, act.K // 2, dtype=torch.uint8, device=act.device)
+    scales = torch.empty(act.M, act.K // 16, dtype=torch.uint8, device=act.device)
+    with torch.cuda.device(act.device):
+        _check("svdq_export_act", lib().svdq_export_act(byref(act.desc), _ptr(codes), _ptr(scales),
+                                                        _stream(act.device)))
+    return codes, scales
+
+
+def device_status(reset: bool = True) -> int:
+    """Synchronizes; returns 0, or the SVDQ_ERR_TIMEOUT status if a bounded device wait ran out."""
+    return lib().svdq_device_status(1 if reset else 0)
+
+
+def watchdog_selftest(limit_ns: int, device=None):
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(device):
+        _check("svdq_watchdog_selftest", lib().svdq_watchdog_selftest(limit_ns, _stream(device)))
+
+
+def set_wait_limit_ns(ns: int):
+    _check("svdq_set_wait_limit_ns", lib().svdq_set_wait_limit_ns(ns))
+
+
+def last_error() -> str:
+    return lib().svdq_last_error().decode()

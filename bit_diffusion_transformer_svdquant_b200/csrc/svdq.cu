@@ -1,0 +1,467 @@
+// C ABI of the sm_100a W4A4 + low-rank linear layer (declared in include/svdq.h): argument checks,
+// buffer layouts, TMA descriptor construction and kernel launches. One translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdlib>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "svdq.h"
+#include "svdq_gemm.cuh"
+#include "svdq_ptx.cuh"
+#include "svdq_quant.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_wait_ns{2000000000ull};
+
+svdq_status fail(svdq_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+svdq_status fail(svdq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define SVDQ_CUDA(call)                                                                         \
+  do {                                                                                          \
+    cudaError_t e_ = (call);                                                                    \
+    if (e_ != cudaSuccess) return fail(SVDQ_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ per-device state
+struct DeviceState {
+  bool ready = false;
+  int sm_count = 0;
+  svdq_status status = SVDQ_OK;
+  std::string error;
+};
+std::mutex g_dev_mu;
+DeviceState g_dev[64];
+
+constexpr int kStagesTile192 = 4;
+constexpr int kStagesTile128 = 5;
+
+using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                            const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                            CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+Encode g_encode = nullptr;
+
+svdq_status device_ready(int* dev_out, int* sm_out) {
+  int dev = 0;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(SVDQ_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0, sms = 0;
+    SVDQ_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    SVDQ_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    SVDQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    if (major != 10 || minor != 0)
+      return fail(SVDQ_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", dev, major,
+                  minor);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      SVDQ_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (fn == nullptr || q != cudaDriverEntryPointSuccess)
+        return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+      g_encode = reinterpret_cast<Encode>(fn);
+    }
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<192, kStagesTile192>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::GemmLayout<192, kStagesTile192>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<128, kStagesTile128>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::GemmLayout<128, kStagesTile128>::kSmem));
+    st.sm_count = sms;
+    st.ready = true;
+  }
+  if (dev_out) *dev_out = dev;
+  if (sm_out) *sm_out = st.sm_count;
+  return SVDQ_OK;
+}
+
+svdq_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SVDQ_OK;
+}
+
+CUtensorMapSwizzle lr_swizzle(int r) {
+  return r == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : (r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool valid_r(int r) { return r == 0 || r == 16 || r == 32 || r == 64; }
+
+int choose_n_tile(int N) {
+  const char* env = getenv("SVDQ_N_TILE");
+  if (env != nullptr) {
+    const int t = atoi(env);
+    if ((t == 128 || t == 192) && N % t == 0) return t;
+  }
+  if (N % 192 == 0) return 192;
+  if (N % 128 == 0) return 128;
+  return 0;
+}
+
+struct WeightLayout {
+  size_t codes, scales, gw, inv_lambda, l1t, l2t, total;
+};
+WeightLayout weight_layout(int N, int K, int r, int n_tile) {
+  WeightLayout l{};
+  size_t off = 0;
+  l.codes = off;
+  off = align_up(off + static_cast<size_t>(N) * K / 2);
+  l.scales = off;
+  off = align_up(off + static_cast<size_t>(N / n_tile) * (K / 64) * ((n_tile + 127) / 128) * 512);
+  l.gw = off;
+  off = align_up(off + 4);
+  l.inv_lambda = off;
+  off = align_up(off + static_cast<size_t>(K) * 4);
+  l.l1t = off;
+  off = align_up(off + static_cast<size_t>(r) * K * 2);
+  l.l2t = off;
+  off = align_up(off + static_cast<size_t>(N) * r * 2);
+  l.total = off;
+  return l;
+}
+
+struct ActLayout {
+  size_t codes, scales, u, alpha, total;
+  int M_pad;
+};
+ActLayout act_layout(int M, int K, int r) {
+  ActLayout l{};
+  l.M_pad = (M + 127) / 128 * 128;
+  size_t off = 0;
+  l.codes = off;
+  off = align_up(off + static_cast<size_t>(l.M_pad) * K / 2);
+  l.scales = off;
+  off = align_up(off + static_cast<size_t>(l.M_pad / 128) * (K / 64) * 512);
+  l.u = off;
+  off = align_up(off + static_cast<size_t>(l.M_pad) * r * 2);
+  l.alpha = off;
+  off = align_up(off + 4);
+  l.total = off;
+  return l;
+}
+
+bool shape_ok(int N, int K, int r) {
+  return N > 0 && K > 0 && K % 256 == 0 && valid_r(r) && K <= (1 << 20) && N <= (1 << 20) && choose_n_tile(N) > 0;
+}
+
+int grid_for(size_t work_items, int per_block, int sm_count) {
+  size_t blocks = (work_items + per_block - 1) / per_block;
+  size_t cap = static_cast<size_t>(sm_count) * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return static_cast<int>(blocks);
+}
+
+svdq_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int svdq_abi_version(void) { return SVDQ_ABI_VERSION; }
+
+const char* svdq_status_str(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_UNSUPPORTED: return "unsupported shape, alignment or device";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* svdq_last_error(void) { return g_last_error.c_str(); }
+
+size_t svdq_weight_bytes(int N, int K, int r) {
+  if (!shape_ok(N, K, r)) return 0;
+  return weight_layout(N, K, r, choose_n_tile(N)).total;
+}
+
+size_t svdq_act_bytes(int M, int K, int r) {
+  if (M < 1 || M >= (1 << 24) || K <= 0 || K % 256 != 0 || !valid_r(r)) return 0;
+  return act_layout(M, K, r).total;
+}
+
+svdq_status svdq_set_wait_limit_ns(unsigned long long ns) {
+  if (ns < 1000000ull || ns > 60000000000ull) return fail(SVDQ_ERR_INVALID_ARG, "wait limit %llu ns out of range", ns);
+  g_wait_ns.store(ns);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_act_bind(int M, int K, int r, void* dst, size_t dst_bytes, svdq_act* out) {
+  if (out == nullptr || dst == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const size_t need = svdq_act_bytes(M, K, r);
+  if (need == 0) return fail(SVDQ_ERR_UNSUPPORTED, "act shape M=%d K=%d r=%d unsupported", M, K, r);
+  if (dst_bytes < need) return fail(SVDQ_ERR_INVALID_ARG, "act buffer %zu bytes < %zu", dst_bytes, need);
+  if (reinterpret_cast<uintptr_t>(dst) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "act buffer not 256-byte aligned");
+  const ActLayout l = act_layout(M, K, r);
+  uint8_t* b = static_cast<uint8_t*>(dst);
+  out->M = M;
+  out->K = K;
+  out->r = r;
+  out->M_pad = l.M_pad;
+  out->codes = b + l.codes;
+  out->scales = b + l.scales;
+  out->U = b + l.u;
+  out->alpha = reinterpret_cast<float*>(b + l.alpha);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const uint16_t* L2_rn,
+                             const float* inv_lambda, int N, int K, int r, int swiglu, void* dst, size_t dst_bytes,
+                             svdq_weight* out, svdq_stream_t stream) {
+  if (out == nullptr || R_nk == nullptr || inv_lambda == nullptr || dst == nullptr)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (r > 0 && (L1s_kr == nullptr || L2_rn == nullptr)) return fail(SVDQ_ERR_INVALID_ARG, "null L1s / L2 with r > 0");
+  if (!shape_ok(N, K, r)) return fail(SVDQ_ERR_UNSUPPORTED, "weight shape N=%d K=%d r=%d unsupported", N, K, r);
+  if (swiglu && (N % 2 != 0)) return fail(SVDQ_ERR_UNSUPPORTED, "SwiGLU needs N even");
+  if (!aligned16(R_nk) || !aligned16(inv_lambda) || (r > 0 && (!aligned16(L1s_kr) || !aligned16(L2_rn))))
+    return fail(SVDQ_ERR_UNSUPPORTED, "inputs must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(dst) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "dst not 256-byte aligned");
+  const int n_tile = choose_n_tile(N);
+  const WeightLayout l = weight_layout(N, K, r, n_tile);
+  if (dst_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "weight buffer %zu bytes < %zu", dst_bytes, l.total);
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* b = static_cast<uint8_t*>(dst);
+
+  svdq_weight w{};
+  w.N = N;
+  w.K = K;
+  w.r = r;
+  w.swiglu_interleaved = swiglu ? 1 : 0;
+  w.n_tile = n_tile;
+  w.codes = b + l.codes;
+  w.scales = b + l.scales;
+  w.g_w = reinterpret_cast<float*>(b + l.gw);
+  w.inv_lambda = reinterpret_cast<float*>(b + l.inv_lambda);
+  w.L1s_t = b + l.l1t;
+  w.L2_t = b + l.l2t;
+
+  SVDQ_CUDA(cudaMemsetAsync(b + l.scales, 0, l.gw - l.scales + 4, st));  // pad rows of the scale layout, amax
+  SVDQ_CUDA(cudaMemcpyAsync(w.inv_lambda, inv_lambda, static_cast<size_t>(K) * 4, cudaMemcpyDeviceToDevice, st));
+  const size_t n4 = static_cast<size_t>(N) * K / 4;
+  svdq::amax_f32_kernel<<<grid_for(n4, 256, sms), 256, 0, st>>>(R_nk, n4, reinterpret_cast<unsigned*>(w.g_w));
+  if (svdq_status s = check_launch("amax_f32_kernel"); s != SVDQ_OK) return s;
+  svdq::finalize_scale_kernel<<<1, 1, 0, st>>>(w.g_w);
+  if (svdq_status s = check_launch("finalize_scale_kernel"); s != SVDQ_OK) return s;
+  const size_t halves = static_cast<size_t>(N) * K / 8;
+  svdq::pack_quant_kernel<<<grid_for(halves, 256, sms), 256, 0, st>>>(
+      R_nk, N, K, n_tile, w.swiglu_interleaved, w.g_w, static_cast<uint8_t*>(w.codes), static_cast<uint8_t*>(w.scales));
+  if (svdq_status s = check_launch("pack_quant_kernel"); s != SVDQ_OK) return s;
+  if (r > 0) {
+    svdq::transpose_l1_kernel<<<grid_for(static_cast<size_t>(K) * r, 256, sms), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(L1s_kr), K, r, static_cast<__nv_bfloat16*>(w.L1s_t));
+    if (svdq_status s = check_launch("transpose_l1_kernel"); s != SVDQ_OK) return s;
+    svdq::pack_l2_kernel<<<grid_for(static_cast<size_t>(N) * r, 256, sms), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(L2_rn), N, r, n_tile, w.swiglu_interleaved,
+        static_cast<__nv_bfloat16*>(w.L2_t));
+    if (svdq_status s = check_launch("pack_l2_kernel"); s != SVDQ_OK) return s;
+  }
+  static_assert(sizeof(w.tmap) >= 2 * sizeof(CUtensorMap), "tmap storage");
+  CUtensorMap tmB, tmL2;
+  std::memset(&tmL2, 0, sizeof(tmL2));
+  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K / 2, N, K / 2, 128, n_tile,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, N, static_cast<uint64_t>(r) * 2,
+                                  r, n_tile, lr_swizzle(r));
+        s != SVDQ_OK)
+      return s;
+  }
+  std::memcpy(&w.tmap[0][0], &tmB, sizeof(CUtensorMap));
+  std::memcpy(&w.tmap[1][0], &tmL2, sizeof(CUtensorMap));
+  *out = w;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_calibrate_act(const uint16_t* X, int M, const svdq_weight* w, float* g_x_out, svdq_stream_t stream) {
+  if (X == nullptr || w == nullptr || g_x_out == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (M < 1 || M >= (1 << 24)) return fail(SVDQ_ERR_UNSUPPORTED, "M=%d unsupported", M);
+  if (!aligned16(X)) return fail(SVDQ_ERR_UNSUPPORTED, "X must be 16-byte aligned");
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SVDQ_CUDA(cudaMemsetAsync(g_x_out, 0, 4, st));
+  const size_t n8 = static_cast<size_t>(M) * w->K / 8;
+  svdq::act_amax_kernel<<<grid_for(n8, 256, sms), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(X),
+                                                                 w->inv_lambda, n8, w->K,
+                                                                 reinterpret_cast<unsigned*>(g_x_out));
+  if (svdq_status s = check_launch("act_amax_kernel"); s != SVDQ_OK) return s;
+  svdq::finalize_scale_kernel<<<1, 1, 0, st>>>(g_x_out);
+  return check_launch("finalize_scale_kernel");
+}
+
+svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const float* g_x, const svdq_act* act,
+                              svdq_stream_t stream) {
+  if (X == nullptr || w == nullptr || g_x == nullptr || act == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (act->K != w->K || act->r != w->r)
+    return fail(SVDQ_ERR_INVALID_ARG, "act (K=%d r=%d) does not match weight (K=%d r=%d)", act->K, act->r, w->K, w->r);
+  if (!aligned16(X)) return fail(SVDQ_ERR_UNSUPPORTED, "X must be 16-byte aligned");
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  svdq::QuantActArgs a;
+  a.X = reinterpret_cast<const __nv_bfloat16*>(X);
+  a.inv_lambda = w->inv_lambda;
+  a.L1s_t = static_cast<const __nv_bfloat16*>(w->L1s_t);
+  a.g_x = g_x;
+  a.g_w = w->g_w;
+  a.codes = static_cast<uint8_t*>(act->codes);
+  a.sf = static_cast<uint8_t*>(act->scales);
+  a.U = static_cast<__nv_bfloat16*>(act->U);
+  a.alpha = act->alpha;
+  a.M = act->M;
+  a.K = act->K;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int grid = act->M_pad / 16;
+  switch (w->r) {
+    case 0: svdq::quant_act_kernel<0><<<grid, 256, 0, st>>>(a); break;
+    case 16: svdq::quant_act_kernel<16><<<grid, 256, 0, st>>>(a); break;
+    case 32: svdq::quant_act_kernel<32><<<grid, 256, 0, st>>>(a); break;
+    case 64: svdq::quant_act_kernel<64><<<grid, 256, 0, st>>>(a); break;
+    default: return fail(SVDQ_ERR_UNSUPPORTED, "r=%d unsupported", w->r);
+  }
+  return check_launch("quant_act_kernel");
+}
+
+svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t* bias, svdq_epilogue epi, void* Y,
+                      svdq_out_dtype out_dtype, svdq_stream_t stream) {
+  if (act == nullptr || w == nullptr || Y == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (act->K != w->K || act->r != w->r) return fail(SVDQ_ERR_INVALID_ARG, "act does not match weight");
+  if (epi < SVDQ_EPI_NONE || epi > SVDQ_EPI_BIAS_SWIGLU) return fail(SVDQ_ERR_INVALID_ARG, "bad epilogue %d", epi);
+  if (out_dtype != SVDQ_OUT_BF16 && out_dtype != SVDQ_OUT_F32) return fail(SVDQ_ERR_INVALID_ARG, "bad out dtype");
+  const bool has_bias = (epi & 1) != 0, swiglu = (epi & 2) != 0;
+  if (has_bias && bias == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "epilogue needs a bias");
+  if (swiglu && !w->swiglu_interleaved) return fail(SVDQ_ERR_INVALID_ARG, "SwiGLU needs a weight packed with swiglu=1");
+  if (!swiglu && w->swiglu_interleaved) return fail(SVDQ_ERR_INVALID_ARG, "weight packed for SwiGLU");
+  if (!aligned16(Y) || (bias != nullptr && !aligned16(bias))) return fail(SVDQ_ERR_UNSUPPORTED, "Y / bias alignment");
+  const int n_tile = w->n_tile;
+  if ((n_tile != 192 && n_tile != 128) || w->N % n_tile != 0) return fail(SVDQ_ERR_UNSUPPORTED, "bad n_tile");
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+
+  const int K = w->K, r = w->r;
+  CUtensorMap tmA, tmU;
+  std::memset(&tmU, 0, sizeof(tmU));
+  if (svdq_status s = make_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, act->codes, K / 2, act->M_pad, K / 2, 128, 128,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act->U, r, act->M_pad,
+                                  static_cast<uint64_t>(r) * 2, r, 128, lr_swizzle(r));
+        s != SVDQ_OK)
+      return s;
+  }
+  CUtensorMap tmB, tmL2;  // properly aligned copies of the descriptors cached in the weight
+  std::memcpy(&tmB, &w->tmap[0][0], sizeof(CUtensorMap));
+  std::memcpy(&tmL2, &w->tmap[1][0], sizeof(CUtensorMap));
+
+  svdq::GemmArgs g{};
+  g.sfa = static_cast<const uint8_t*>(act->scales);
+  g.sfb = static_cast<const uint8_t*>(w->scales);
+  g.alpha = act->alpha;
+  g.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  g.Y = Y;
+  g.wait_ns = g_wait_ns.load();
+  g.M = act->M;
+  g.N = w->N;
+  g.K = K;
+  g.r = r;
+  g.m_tiles = act->M_pad / 128;
+  g.n_tiles = w->N / n_tile;
+  g.k_iters = K / 256;
+  g.num_tiles = g.m_tiles * g.n_tiles;
+  g.ldy = swiglu ? w->N / 2 : w->N;
+  g.out_f32 = out_dtype == SVDQ_OUT_F32 ? 1 : 0;
+  g.epi = static_cast<int>(epi);
+  const int grid = g.num_tiles < sms ? g.num_tiles : sms;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_tile == 192) {
+    svdq::svdq_gemm_kernel<192, kStagesTile192><<<grid, 192, svdq::GemmLayout<192, kStagesTile192>::kSmem, st>>>(
+        tmA, tmB, tmU, tmL2, g);
+  } else {
+    svdq::svdq_gemm_kernel<128, kStagesTile128><<<grid, 192, svdq::GemmLayout<128, kStagesTile128>::kSmem, st>>>(
+        tmA, tmB, tmU, tmL2, g);
+  }
+  return check_launch("svdq_gemm_kernel");
+}
+
+svdq_status svdq_export_weight(const svdq_weight* w, uint8_t* codes, uint8_t* scales, svdq_stream_t stream) {
+  if (w == nullptr || codes == nullptr || scales == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  const size_t total = static_cast<size_t>(w->N) * (w->K / 16);
+  svdq::export_weight_kernel<<<grid_for(total, 256, sms), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->scales), w->N, w->K, w->n_tile,
+      w->swiglu_interleaved, codes, scales);
+  return check_launch("export_weight_kernel");
+}
+
+svdq_status svdq_export_act(const svdq_act* act, uint8_t* codes, uint8_t* scales, svdq_stream_t stream) {
+  if (act == nullptr || codes == nullptr || scales == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  const size_t total = static_cast<size_t>(act->M) * (act->K / 16);
+  svdq::export_act_kernel<<<grid_for(total, 256, sms), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(act->codes), static_cast<const uint8_t*>(act->scales), act->M, act->K, codes,
+      scales);
+  return check_launch("export_act_kernel");
+}
+
+svdq_status svdq_device_status(int reset) {
+  SVDQ_CUDA(cudaDeviceSynchronize());
+  unsigned v = 0;
+  SVDQ_CUDA(cudaMemcpyFromSymbol(&v, svdq::g_svdq_status, sizeof(v)));
+  if (reset) {
+    const unsigned z = 0;
+    SVDQ_CUDA(cudaMemcpyToSymbol(svdq::g_svdq_status, &z, sizeof(z)));
+  }
+  if (v != 0) return fail(SVDQ_ERR_TIMEOUT, "device wait ran out (status bits 0x%x)", v);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_watchdog_selftest(unsigned long long limit_ns, svdq_stream_t stream) {
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull) return fail(SVDQ_ERR_INVALID_ARG, "limit out of range");
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  svdq::watchdog_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return check_launch("watchdog_selftest_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,346 @@
+// Kernel 2: block-scaled NVFP4 GEMM on the 5th-generation tensor cores (tcgen05), with the
+// low-rank up-projection and the bias / SwiGLU epilogue fused in.
+//
+// Method ("Bringing Nunchaku 4-bit diffusion inference to Diffusers", "SVDQuant deep dive"): the
+// branch's up-projection (X L1) L2 is fused with the 4-bit GEMM; here it is one extra bf16 MMA
+// (K = r) into the same TMEM accumulator, with U pre-divided by alpha = g_x g_w so that a single
+// scale applies at the end. The fused QKV / SwiGLU epilogues follow the fused NVFP4 GEMMs of
+// "FLUX 3 Image Klein on NVIDIA Blackwell", method 1.
+//
+// Structure (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: per 256-wide K step, A (128 x 128 B) and B (n_tile x 128 B) codes as
+//               128B-swizzled 2-D tiles, plus the matching scale-factor atoms as 1-D bulk copies,
+//               into a STAGES-deep shared-memory ring (full/empty mbarriers). Before a tile's K
+//               loop, one ring slot carries the tile's U (128 x r) and L2^T (n_tile x r) bf16.
+//   warp 1      TMEM allocator + single-thread MMA issuer: tcgen05.cp of the scale factors into
+//               TMEM, 4 x tcgen05.mma kind::mxf4nvf4 (M=128, N=n_tile, K=64) per K step, r/16 x
+//               kind::f16 for the low-rank term; tcgen05.commit frees ring slots and publishes
+//               finished accumulators. Accumulators are double-buffered in TMEM when they fit.
+//   warps 2..5  epilogue: tcgen05.ld (each warp its 32-lane quadrant), y = alpha acc (+ bias),
+//               SwiGLU on interleaved gate/up columns, bf16 or fp32 store.
+// Every mbarrier wait is bounded (global timer); a wait that runs out records a status bit, sets
+// a shared abort flag so that the other roles stop too, and the kernel drains its own copies and
+// MMAs before freeing TMEM and returning.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "svdq_ptx.cuh"
+#include "svdq_quant.cuh"
+
+namespace svdq {
+
+struct GemmArgs {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* alpha;
+  const __nv_bfloat16* bias;
+  void* Y;
+  unsigned long long wait_ns;
+  int M, N, K, r;
+  int m_tiles, n_tiles, k_iters, num_tiles;
+  int ldy, out_f32, epi;  // epi bit 0: bias, bit 1: SwiGLU
+};
+
+template <int N_TILE, int STAGES>
+struct GemmLayout {
+  static constexpr int kA = 128 * 128;
+  static constexpr int kB = N_TILE * 128;
+  static constexpr int kSfAtomsB = (N_TILE + 127) / 128;
+  static constexpr int kSfa = 4 * 512;
+  static constexpr int kSfb = 4 * kSfAtomsB * 512;
+  static constexpr int kStage = kA + kB + kSfa + kSfb;
+  static constexpr int kOffB = kA;
+  static constexpr int kOffSfa = kA + kB;
+  static constexpr int kOffSfb = kA + kB + kSfa;
+  static constexpr int kSfCols = 16 + 16 * kSfAtomsB;
+  static constexpr int kAccBufs = (2 * N_TILE + kSfCols <= 512) ? 2 : 1;
+  static constexpr int kColSfa = kAccBufs * N_TILE;
+  static constexpr int kColSfb = kColSfa + 16;
+  static constexpr int kBarOff = STAGES * kStage;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1;
+  static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
+  static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kColSfb + 16 * kSfAtomsB <= 512, "TMEM budget");
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ uint32_t lr_swizzle_mode(int r) { return r == 16 ? 6u : (r == 32 ? 4u : 2u); }
+
+template <int N_TILE, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    svdq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
+                     const GemmArgs args) {
+  using L = GemmLayout<N_TILE, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kAccBufs + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * L::kAccBufs);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = args.r;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < L::kAccBufs; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if (r > 0) {
+      prefetch_tmap(&tmU);
+      prefetch_tmap(&tmL2);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  unsigned* status = &g_svdq_status;
+  const uint64_t wait_ns = args.wait_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
+      const uint32_t lr_bytes = static_cast<uint32_t>((128 + N_TILE) * r * 2);
+      const int sf_row_stride = args.K >> 6;  // 64-wide K atoms per 128-row block
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+        const int m_blk = tile % args.m_tiles, n_blk = tile / args.m_tiles;
+        if (r > 0) {
+          if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
+            break;
+          const uint32_t sa = sbase + stage * L::kStage;
+          mbar_arrive_expect_tx(full_bar(stage), lr_bytes);
+          tma_load_2d(sa, &tmU, 0, m_blk * 128, full_bar(stage));
+          tma_load_2d(sa + L::kOffB, &tmL2, 0, n_blk * N_TILE, full_bar(stage));
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        const uint8_t* sfa_tile = args.sfa + (static_cast<size_t>(m_blk) * sf_row_stride << 9);
+        const uint8_t* sfb_tile = args.sfb + (static_cast<size_t>(n_blk) * sf_row_stride * L::kSfAtomsB << 9);
+        for (int kt = 0; kt < args.k_iters; ++kt) {
+          if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
+            break;
+          const uint32_t sa = sbase + stage * L::kStage;
+          mbar_arrive_expect_tx(full_bar(stage), L::kStage);
+          tma_load_2d(sa, &tmA, kt * 128, m_blk * 128, full_bar(stage));
+          tma_load_2d(sa + L::kOffB, &tmB, kt * 128, n_blk * N_TILE, full_bar(stage));
+          bulk_load(sa + L::kOffSfa, sfa_tile + (static_cast<size_t>(kt) * 4 << 9), L::kSfa, full_bar(stage));
+          bulk_load(sa + L::kOffSfb, sfb_tile + (static_cast<size_t>(kt) * 4 * L::kSfAtomsB << 9), L::kSfb,
+                    full_bar(stage));
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Drain: every copy this thread started has landed before the CTA may exit.
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s))
+          mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      const uint32_t idesc_fp4 = idesc_nvfp4(128, N_TILE);
+      const uint32_t idesc_lr = idesc_bf16(128, N_TILE);
+      const uint32_t lr_swz = lr_swizzle_mode(r);
+      const uint32_t lr_sbo = 8u * r * 2u;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+        if (!(ok = mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, wait_ns, status, kStatusMma, abort_flag)))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
+        uint32_t accumulate = 0;
+        if (r > 0) {
+          if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * L::kStage;
+          const uint64_t du = smem_desc(sa, 16, lr_sbo, lr_swz);
+          const uint64_t dl = smem_desc(sa + L::kOffB, 16, lr_sbo, lr_swz);
+          for (int j = 0; j < (r >> 4); ++j) {
+            mma_bf16(d, du + 2u * j, dl + 2u * j, idesc_lr, accumulate);
+            accumulate = 1;
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        for (int kt = 0; kt < args.k_iters; ++kt) {
+          if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * L::kStage;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            tc_cp_sf(tmem + L::kColSfa + 4 * i, smem_desc(sa + L::kOffSfa + 512 * i, 0, 128, 0));
+#pragma unroll
+          for (int i = 0; i < 4 * L::kSfAtomsB; ++i)
+            tc_cp_sf(tmem + L::kColSfb + 4 * i, smem_desc(sa + L::kOffSfb + 512 * i, 0, 128, 0));
+          const uint64_t da = smem_desc(sa, 16, 1024, 2);
+          const uint64_t db = smem_desc(sa + L::kOffB, 16, 1024, 2);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            mma_nvfp4(d, da + 2u * i, db + 2u * i, idesc_fp4, tmem + L::kColSfa + 4 * i,
+                      tmem + L::kColSfb + 4 * L::kSfAtomsB * i, accumulate);
+            accumulate = 1;
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(acc));
+        if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+      }
+      // Drain: all issued MMAs and scale copies complete before TMEM is freed.
+      tc_commit(drain_bar);
+      mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    const float alpha = *args.alpha;
+    const bool has_bias = (args.epi & 1) != 0;
+    const bool swiglu = (args.epi & 2) != 0;
+    const int hN = args.N >> 1;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+      const int m_blk = tile % args.m_tiles, n_blk = tile / args.m_tiles;
+      // warp-uniform outcome: tcgen05.ld below is a .sync.aligned warp instruction
+      const bool got = mbar_wait_bounded(accf_bar(acc), acc_phase, wait_ns, status, kStatusEpilogue, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int row = m_blk * 128 + q * 32 + lane;
+      const bool row_ok = row < args.M;
+      const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * N_TILE);
+      if (!swiglu) {
+#pragma unroll 1
+        for (int c = 0; c < N_TILE / 32; ++c) {
+          float v[32];
+          tmem_ld_32x32(tb + c * 32, v);
+          tmem_wait_ld();
+          const int n0 = n_blk * N_TILE + c * 32;
+          if (has_bias) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              float b[8];
+              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n0 + i)), b);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) v[i + j] = fmaf(alpha, v[i + j], b[j]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = alpha * v[i];
+          }
+          if (row_ok) {
+            if (args.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + static_cast<size_t>(row) * args.ldy + n0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + static_cast<size_t>(row) * args.ldy + n0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint32_t w[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
+                  w[j] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
+        }
+      } else {
+        constexpr int kHalf = N_TILE / 2;
+#pragma unroll 1
+        for (int c = 0; c < kHalf / 32; ++c) {
+          float gt[32], up[32];
+          tmem_ld_32x32(tb + c * 32, gt);
+          tmem_ld_32x32(tb + kHalf + c * 32, up);
+          tmem_wait_ld();
+          const int j0 = n_blk * kHalf + c * 32;
+          if (has_bias) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              float bg[8], bu[8];
+              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + j0 + i)), bg);
+              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + hN + j0 + i)), bu);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                gt[i + j] = fmaf(alpha, gt[i + j], bg[j]);
+                up[i + j] = fmaf(alpha, up[i + j], bu[j]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              gt[i] = alpha * gt[i];
+              up[i] = alpha * up[i];
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) gt[i] = gt[i] / (1.0f + __expf(-gt[i])) * up[i];
+          if (row_ok) {
+            if (args.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + static_cast<size_t>(row) * args.ldy + j0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dst[i] = make_float4(gt[4 * i], gt[4 * i + 1], gt[4 * i + 2], gt[4 * i + 3]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + static_cast<size_t>(row) * args.ldy + j0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint32_t w[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const __nv_bfloat162 h = __floats2bfloat162_rn(gt[8 * i + 2 * j], gt[8 * i + 2 * j + 1]);
+                  w[j] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace svdq

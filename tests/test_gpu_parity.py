@@ -1,0 +1,130 @@
+"""GPU parity: the CUDA path (through the C ABI) against the oracle on the same seeded inputs.
+
+Bar: tensor scales, E2M1 codes and E4M3 scales bit-exact; fp32 outputs within
+max|y - y_ref| <= 2e-3 * max|y_ref|; bf16 outputs bitwise equal to the bf16 rounding of the fp32
+outputs; repeated runs bitwise identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_diffusion_transformer_svdquant_b200 as svdq
+from bit_diffusion_transformer_svdquant_b200 import synth
+from oracle import nvfp4, svdquant
+
+from _parity import Case
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand_layer(M, K, N, r, seed, bias=True, outlier=50.0):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((M, K))
+    X[:, rng.choice(K, max(1, K // 100), replace=False)] *= outlier
+    X = svdquant.bf16_round(X)
+    W = svdquant.bf16_round(rng.standard_normal((N, K)) / np.sqrt(K))
+    b = svdquant.bf16_round(rng.standard_normal(N) * np.sqrt(0.02)) if bias else None
+    return X, W, b
+
+
+def test_watchdog_selftest_returns_status(cuda_device):
+    assert svdq.device_status(reset=True) == 0
+    svdq.watchdog_selftest(2_000_000, cuda_device)       # 2 ms wait that nothing ends
+    assert svdq.device_status(reset=True) == 4            # SVDQ_ERR_TIMEOUT, context still usable
+    assert svdq.device_status(reset=True) == 0
+    x = torch.ones(4, device=cuda_device)
+    assert float(x.sum().item()) == 4.0
+
+
+def test_codec_edges_through_kernel1(cuda_device):
+    """Hand-built blocks that land exactly on E2M1 and E4M3 rounding ties, E4M3 subnormal and zero
+    scales, saturation and signed zeros, pushed through the activation kernel with lambda = 1 and a
+    static g_x = 1 (so that block values reach the codecs unscaled; row 2 exceeds the calibrated
+    range and saturates)."""
+    K, M = 256, 32
+    rng = np.random.default_rng(11)
+    X = svdquant.bf16_round(rng.standard_normal((M, K)))
+    X[1, 0:16] = [6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5, -5, -0.1015625]
+    X[1, 16:32] = [6.375] + [1.0] * 15                   # amax/6 = 1.0625: E4M3 tie -> 1.0
+    X[1, 32:48] = [7.125] + [-0.5] * 15                  # amax/6 = 1.1875: tie -> 1.25
+    X[1, 48:64] = [6 * 2.0 ** -10] + [1e-4] * 15         # amax/6 = 2^-10: tie -> 0 -> zero block
+    X[1, 64:80] = [6 * 1.5 * 2.0 ** -9] + [0.001] * 15   # tie between 1 and 2 subnormal steps -> 2
+    X[1, 80:96] = 0.0
+    X[1, 96:112] = -0.0
+    X[2, :] = svdquant.bf16_round(rng.standard_normal(K) * 1e4)   # saturating scales and codes
+    X = svdquant.bf16_round(X)
+    W = svdquant.bf16_round(rng.standard_normal((128, K)) / 16)
+    prep = {"inv_lambda": np.ones(K), "lam_prime": np.ones(K), "L1s": np.zeros((K, 0)), "L2": np.zeros((0, 128)),
+            "R": nvfp4.f32(W), "r": 0}
+    c = Case(X, W, None, 0, False, cuda_device, prep=prep, g_x=1.0)
+    c.check_scales()
+    c.check_act_codes()
+    c.check_weight_codes()
+    c.check_outputs()
+
+
+SMALL_CASES = [
+    # M, K, N, r, bias, swiglu
+    (300, 768, 384, 32, True, False),   # ragged M, two 192-wide tiles
+    (1, 256, 128, 0, False, False),     # one row, no low-rank branch, 128-wide tile
+    (200, 512, 768, 64, True, True),    # SwiGLU with bias, r = 64
+    (130, 1024, 256, 16, False, True),  # SwiGLU, no bias, 128-wide tile
+    (513, 256, 192, 32, False, False),  # a ragged fifth m-tile, K = one k-step
+    (1000, 2048, 1152, 32, True, False),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,bias,swiglu", SMALL_CASES)
+def test_small_shapes(cuda_device, M, K, N, r, bias, swiglu):
+    X, W, b = _rand_layer(M, K, N, r, seed=M * 7 + N, bias=bias)
+    c = Case(X, W, b, r, swiglu, cuda_device)
+    c.check_scales()
+    c.check_weight_codes()
+    c.check_act_codes()
+    c.check_outputs()
+
+
+def test_tiny_workload(cuda_device):
+    spec = synth.WORKLOADS["tiny"].layers[0]
+    d = synth.make_linear_inputs(spec)
+    c = Case(synth.bf16_values(d["X"]), synth.bf16_values(d["W"]), None, spec.r, False, cuda_device)
+    c.check_scales()
+    c.check_weight_codes()
+    c.check_act_codes()
+    c.check_outputs()
+
+
+def test_repeatable(cuda_device):
+    X, W, b = _rand_layer(384, 512, 384, 32, seed=5)
+    c = Case(X, W, b, 32, False, cuda_device)
+    y1 = c.run_gemm(torch.float32).clone()
+    u1 = c.act.U().clone()
+    svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
+    y2 = c.run_gemm(torch.float32)
+    assert torch.equal(u1, c.act.U())
+    assert torch.equal(y1, y2)
+
+
+def _full_layers():
+    out = []
+    for wl in synth.WORKLOADS.values():
+        if wl.name == "tiny":
+            continue
+        for spec in wl.layers:
+            out.append(pytest.param(spec, id=spec.name))
+    return out
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("spec", _full_layers())
+def test_full_size_workload(cuda_device, spec):
+    """Every layer of every workload at its full size: all codes and scales bit-exact, outputs on a
+    few thousand sampled positions (plus tile corners and the last row) within tolerance."""
+    d = synth.make_linear_inputs(spec)
+    X, W = synth.bf16_values(d["X"]), synth.bf16_values(d["W"])
+    b = synth.bf16_values(d["bias"]) if spec.bias else None
+    c = Case(X, W, b, spec.r, spec.swiglu, cuda_device)
+    c.check_scales()
+    c.check_weight_codes()
+    c.check_act_codes()
+    c.check_outputs(samples=3000)
