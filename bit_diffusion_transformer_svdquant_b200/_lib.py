@@ -159,7 +159,9 @@ class QuantizedAct:
         return self.buf[off:off + nbytes]
 
     def U(self) -> torch.Tensor:
-        return self._view(self.desc.U, self.desc.M_pad * self.r * 2).view(torch.bfloat16).view(self.desc.M_pad, self.r)
+        """[2, M_pad, r] bf16: the hi and lo halves of X L1s / alpha."""
+        n = self.desc.M_pad * self.r
+        return self._view(self.desc.U, 2 * n * 2).view(torch.bfloat16).view(2, self.desc.M_pad, self.r)
 
     def alpha(self) -> torch.Tensor:
         return self._view(self.desc.alpha, 4).view(torch.float32)

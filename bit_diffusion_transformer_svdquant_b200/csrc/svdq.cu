@@ -108,9 +108,8 @@ svdq_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, 
   return SVDQ_OK;
 }
 
-CUtensorMapSwizzle lr_swizzle(int r) {
-  return r == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : (r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
-}
+// The low-rank operands travel in chunks of at most 32 columns of r (one ring slot each).
+CUtensorMapSwizzle lr_swizzle(int r) { return r == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B; }
 
 bool valid_r(int r) { return r == 0 || r == 16 || r == 32 || r == 64; }
 
@@ -160,7 +159,7 @@ ActLayout act_layout(int M, int K, int r) {
   l.scales = off;
   off = align_up(off + static_cast<size_t>(l.M_pad / 128) * (K / 64) * 512);
   l.u = off;
-  off = align_up(off + static_cast<size_t>(l.M_pad) * r * 2);
+  off = align_up(off + static_cast<size_t>(l.M_pad) * r * 2 * 2);  // hi and lo halves
   l.alpha = off;
   off = align_up(off + 4);
   l.total = off;
@@ -300,7 +299,7 @@ svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const ui
     return s;
   if (r > 0) {
     if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, N, static_cast<uint64_t>(r) * 2,
-                                  r, n_tile, lr_swizzle(r));
+                                  r < 32 ? r : 32, n_tile, lr_swizzle(r));
         s != SVDQ_OK)
       return s;
   }
@@ -347,6 +346,7 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
   a.alpha = act->alpha;
   a.M = act->M;
   a.K = act->K;
+  a.M_pad = act->M_pad;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int grid = act->M_pad / 16;
   switch (w->r) {
@@ -383,8 +383,8 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
       s != SVDQ_OK)
     return s;
   if (r > 0) {
-    if (svdq_status s = make_tmap(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act->U, r, act->M_pad,
-                                  static_cast<uint64_t>(r) * 2, r, 128, lr_swizzle(r));
+    if (svdq_status s = make_tmap(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act->U, r, 2 * static_cast<uint64_t>(act->M_pad),
+                                  static_cast<uint64_t>(r) * 2, r < 32 ? r : 32, 128, lr_swizzle(r));
         s != SVDQ_OK)
       return s;
   }
@@ -400,6 +400,7 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
   g.Y = Y;
   g.wait_ns = g_wait_ns.load();
   g.M = act->M;
+  g.M_pad = act->M_pad;
   g.N = w->N;
   g.K = K;
   g.r = r;

@@ -11,10 +11,11 @@
 //   warp 0      TMA producer: per 256-wide K step, A (128 x 128 B) and B (n_tile x 128 B) codes as
 //               128B-swizzled 2-D tiles, plus the matching scale-factor atoms as 1-D bulk copies,
 //               into a STAGES-deep shared-memory ring (full/empty mbarriers). Before a tile's K
-//               loop, one ring slot carries the tile's U (128 x r) and L2^T (n_tile x r) bf16.
+//               loop, ring slots carry the tile's U_hi, U_lo (128 x r) and L2^T (n_tile x r) in
+//               chunks of 32 columns of r.
 //   warp 1      TMEM allocator + single-thread MMA issuer: tcgen05.cp of the scale factors into
-//               TMEM, 4 x tcgen05.mma kind::mxf4nvf4 (M=128, N=n_tile, K=64) per K step, r/16 x
-//               kind::f16 for the low-rank term; tcgen05.commit frees ring slots and publishes
+//               TMEM, 4 x tcgen05.mma kind::mxf4nvf4 (M=128, N=n_tile, K=64) per K step, 2 r/16 x
+//               kind::f16 (hi and lo halves of U against the same L2 tile) for the low-rank term; tcgen05.commit frees ring slots and publishes
 //               finished accumulators. Accumulators are double-buffered in TMEM when they fit.
 //   warps 2..5  epilogue: tcgen05.ld (each warp its 32-lane quadrant), y = alpha acc (+ bias),
 //               SwiGLU on interleaved gate/up columns, bf16 or fp32 store.
@@ -38,7 +39,7 @@ struct GemmArgs {
   const __nv_bfloat16* bias;
   void* Y;
   unsigned long long wait_ns;
-  int M, N, K, r;
+  int M, M_pad, N, K, r;
   int m_tiles, n_tiles, k_iters, num_tiles;
   int ldy, out_f32, epi;  // epi bit 0: bias, bit 1: SwiGLU
 };
@@ -66,7 +67,11 @@ struct GemmLayout {
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ uint32_t lr_swizzle_mode(int r) { return r == 16 ? 6u : (r == 32 ? 4u : 2u); }
+// Low-rank operands move in chunks of rc = min(r, 32) columns: U_hi, U_lo (128 x rc each) and
+// L2^T (n_tile x rc), all bf16 with rc*2-byte rows (32B or 64B swizzle), one ring slot per chunk.
+constexpr int kLrChunk = 32;
+constexpr int kOffULo = 128 * kLrChunk * 2;
+__device__ __forceinline__ uint32_t lr_swizzle_mode(int rc) { return rc == 16 ? 6u : 4u; }
 
 template <int N_TILE, int STAGES>
 __global__ void __launch_bounds__(192, 1)
@@ -124,22 +129,25 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
-      const uint32_t lr_bytes = static_cast<uint32_t>((128 + N_TILE) * r * 2);
+      const int rc = r < kLrChunk ? r : kLrChunk;
+      const uint32_t lr_bytes = static_cast<uint32_t>((2 * 128 + N_TILE) * rc * 2);
       const int sf_row_stride = args.K >> 6;  // 64-wide K atoms per 128-row block
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
         const int m_blk = tile % args.m_tiles, n_blk = tile / args.m_tiles;
-        if (r > 0) {
+        for (int c0 = 0; c0 < r; c0 += kLrChunk) {
           if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
             break;
           const uint32_t sa = sbase + stage * L::kStage;
           mbar_arrive_expect_tx(full_bar(stage), lr_bytes);
-          tma_load_2d(sa, &tmU, 0, m_blk * 128, full_bar(stage));
-          tma_load_2d(sa + L::kOffB, &tmL2, 0, n_blk * N_TILE, full_bar(stage));
+          tma_load_2d(sa, &tmU, c0, m_blk * 128, full_bar(stage));
+          tma_load_2d(sa + kOffULo, &tmU, c0, args.M_pad + m_blk * 128, full_bar(stage));
+          tma_load_2d(sa + L::kOffB, &tmL2, c0, n_blk * N_TILE, full_bar(stage));
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        if (!ok) break;
         const uint8_t* sfa_tile = args.sfa + (static_cast<size_t>(m_blk) * sf_row_stride << 9);
         const uint8_t* sfb_tile = args.sfb + (static_cast<size_t>(n_blk) * sf_row_stride * L::kSfAtomsB << 9);
         for (int kt = 0; kt < args.k_iters; ++kt) {
@@ -169,8 +177,9 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0, acc_phase = 0;
       const uint32_t idesc_fp4 = idesc_nvfp4(128, N_TILE);
       const uint32_t idesc_lr = idesc_bf16(128, N_TILE);
-      const uint32_t lr_swz = lr_swizzle_mode(r);
-      const uint32_t lr_sbo = 8u * r * 2u;
+      const int rc = r < kLrChunk ? r : kLrChunk;
+      const uint32_t lr_swz = lr_swizzle_mode(rc);
+      const uint32_t lr_sbo = 8u * rc * 2u;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
         if (!(ok = mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, wait_ns, status, kStatusMma, abort_flag)))
@@ -178,19 +187,22 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
         uint32_t accumulate = 0;
-        if (r > 0) {
+        for (int c0 = 0; c0 < r; c0 += kLrChunk) {
           if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
           tc_fence_after();
           const uint32_t sa = sbase + stage * L::kStage;
-          const uint64_t du = smem_desc(sa, 16, lr_sbo, lr_swz);
+          const uint64_t dhi = smem_desc(sa, 16, lr_sbo, lr_swz);
+          const uint64_t dlo = smem_desc(sa + kOffULo, 16, lr_sbo, lr_swz);
           const uint64_t dl = smem_desc(sa + L::kOffB, 16, lr_sbo, lr_swz);
-          for (int j = 0; j < (r >> 4); ++j) {
-            mma_bf16(d, du + 2u * j, dl + 2u * j, idesc_lr, accumulate);
+          for (int j = 0; j < (rc >> 4); ++j) {
+            mma_bf16(d, dhi + 2u * j, dl + 2u * j, idesc_lr, accumulate);
+            mma_bf16(d, dlo + 2u * j, dl + 2u * j, idesc_lr, 1u);
             accumulate = 1;
           }
           tc_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        if (!ok) break;
         for (int kt = 0; kt < args.k_iters; ++kt) {
           if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
           tc_fence_after();

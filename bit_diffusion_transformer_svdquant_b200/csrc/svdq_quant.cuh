@@ -98,6 +98,8 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
 
 // ------------------------------------------------------------------------------------------------
 // Kernel 1: smoothing + NVFP4 activation quantization + U = X L1s, one pass over X.
+// U is stored divided by alpha = g_x g_w (so the GEMM applies one scale at the end) as a bf16
+// hi/lo pair.
 // CTA = 16 rows x all of K, 8 warps splitting K in 32-column chunks. Within a warp, lane (g, t)
 // (g = lane/4, t = lane%4) loads 8 consecutive bf16 of rows g and g+8 with 128-bit loads; the same
 // registers are both the quantizer's input and the A fragments of two m16n8k16 bf16 MMAs (the
@@ -110,9 +112,9 @@ struct QuantActArgs {
   const float* g_w;
   uint8_t* codes;              // [M_pad][K/2]
   uint8_t* sf;                 // activation MMA layout
-  __nv_bfloat16* U;            // [M_pad][r]
+  __nv_bfloat16* U;            // [2][M_pad][r]: hi then lo
   float* alpha;
-  int M, K;
+  int M, K, M_pad;
 };
 
 template <int R>
@@ -197,12 +199,19 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const QuantActArgs a) {
       pw[(g + 8) * R + col + 1] = acc[j][3];
     }
     __syncthreads();
+    // U / alpha as a bf16 pair: hi = bf16(u), lo = bf16(u - hi) (the difference is exact in fp32),
+    // so that two bf16 MMAs against L2 carry about 16 significant bits of the branch.
     const float cinv = __frcp_rn(alpha);
+    __nv_bfloat16* u_hi = a.U + static_cast<size_t>(m0) * R;
+    __nv_bfloat16* u_lo = u_hi + static_cast<size_t>(a.M_pad) * R;
     for (int i = threadIdx.x; i < 16 * R; i += 256) {
       float s = 0.0f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) s += part[w * 16 * R + i];
-      a.U[static_cast<size_t>(m0) * R + i] = __float2bfloat16_rn(__fmul_rn(s, cinv));
+      const float u = __fmul_rn(s, cinv);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+      u_hi[i] = hi;
+      u_lo[i] = __float2bfloat16_rn(__fsub_rn(u, __bfloat162float(hi)));
     }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.alpha = alpha;

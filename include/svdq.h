@@ -95,7 +95,8 @@ typedef struct svdq_act {
   void* codes;            /* uint8 [M_pad][K/2] E2M1 codes (rows >= M are zero)                */
   void* scales;           /* E4M3, [M_pad/128][K/64] atoms of 512 bytes: byte                  */
                           /*   (m%32)*16 + ((m%128)/32)*4 + (k/16)%4 of atom (m/128, k/64)     */
-  void* U;                /* bf16 [M_pad][r]: bf16(fp32(X L1s) / alpha)                        */
+  void* U;                /* bf16 [2][M_pad][r]: u = fp32(X L1s) / alpha as hi = bf16(u) then  */
+                          /*   lo = bf16(u - hi), ~16 significant bits for the up-projection   */
   float* alpha;           /* device fp32: fp32(g_x * g_w)                                      */
 } svdq_act;
 

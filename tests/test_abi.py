@@ -35,7 +35,7 @@ def test_size_queries(L):
     assert L.svdq_weight_bytes(9216, 3072, 24) == 0          # r not in {0,16,32,64}
     assert L.svdq_weight_bytes(100, 3072, 32) == 0           # N not a multiple of 128 or 192
     na = L.svdq_act_bytes(16896, 3072, 32)
-    assert na >= 16896 * 1536 + 132 * 48 * 512 + 16896 * 32 * 2
+    assert na >= 16896 * 1536 + 132 * 48 * 512 + 2 * 16896 * 32 * 2
     assert L.svdq_act_bytes(0, 3072, 32) == 0
 
 
@@ -47,7 +47,7 @@ def test_act_bind_layout(L):
     assert L.svdq_act_bind(M, K, r, ctypes.c_void_p(base), nb, ctypes.byref(act)) == 0
     assert act.M_pad == 384 and act.codes == base
     assert act.scales - act.codes >= 384 * 256 and act.scales % 256 == 0
-    assert act.U - act.scales >= 3 * 8 * 512 and act.alpha - act.U >= 384 * 16 * 2
+    assert act.U - act.scales >= 3 * 8 * 512 and act.alpha - act.U >= 2 * 384 * 16 * 2
     assert L.svdq_act_bind(M, K, r, ctypes.c_void_p(base), nb - 1, ctypes.byref(act)) == 1
     assert L.svdq_act_bind(M, K, r, ctypes.c_void_p(base + 16), nb, ctypes.byref(act)) == 2
 
