@@ -88,6 +88,14 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<128, kStagesTile128>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<128, kStagesTile128>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<0>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<16>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<32>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<64>::kSmem));
     st.sm_count = sms;
     st.ready = true;
   }
@@ -334,28 +342,69 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
   if (!aligned16(X)) return fail(SVDQ_ERR_UNSUPPORTED, "X must be 16-byte aligned");
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  const int K = act->K, r = w->r, M = act->M;
+  CUtensorMap tmX, tmL1;
+  std::memset(&tmL1, 0, sizeof(tmL1));
+  if (svdq_status s = make_tmap(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(K) * 2, 64, 128,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L1s_t, K, r,
+                                  static_cast<uint64_t>(K) * 2, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+        s != SVDQ_OK)
+      return s;
+  }
+  // K split across a cluster of 1, 2 or 4 CTAs so that small M still fills the SMs
+  const int m_tiles = act->M_pad / 128;
+  int csize = 1;
+  while (csize < 4 && m_tiles * csize < sms && (K / (2 * csize)) % 64 == 0) csize *= 2;
   svdq::QuantActArgs a;
-  a.X = reinterpret_cast<const __nv_bfloat16*>(X);
   a.inv_lambda = w->inv_lambda;
-  a.L1s_t = static_cast<const __nv_bfloat16*>(w->L1s_t);
   a.g_x = g_x;
   a.g_w = w->g_w;
   a.codes = static_cast<uint8_t*>(act->codes);
   a.sf = static_cast<uint8_t*>(act->scales);
   a.U = static_cast<__nv_bfloat16*>(act->U);
   a.alpha = act->alpha;
-  a.M = act->M;
-  a.K = act->K;
+  a.wait_ns = g_wait_ns.load();
+  a.M = M;
+  a.K = K;
   a.M_pad = act->M_pad;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int grid = act->M_pad / 16;
-  switch (w->r) {
-    case 0: svdq::quant_act_kernel<0><<<grid, 256, 0, st>>>(a); break;
-    case 16: svdq::quant_act_kernel<16><<<grid, 256, 0, st>>>(a); break;
-    case 32: svdq::quant_act_kernel<32><<<grid, 256, 0, st>>>(a); break;
-    case 64: svdq::quant_act_kernel<64><<<grid, 256, 0, st>>>(a); break;
-    default: return fail(SVDQ_ERR_UNSUPPORTED, "r=%d unsupported", w->r);
+  a.k_per_cta = K / csize;
+
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(m_tiles * csize, 1, 1);
+  cfg.blockDim = dim3(svdq::kQThreads, 1, 1);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaSuccess;
+  switch (r) {
+    case 0:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<0>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<0>, tmX, tmL1, a);
+      break;
+    case 16:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<16>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<16>, tmX, tmL1, a);
+      break;
+    case 32:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<32>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<32>, tmX, tmL1, a);
+      break;
+    case 64:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<64>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<64>, tmX, tmL1, a);
+      break;
+    default: return fail(SVDQ_ERR_UNSUPPORTED, "r=%d unsupported", r);
   }
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of quant_act_kernel failed: %s", cudaGetErrorString(e));
   return check_launch("quant_act_kernel");
 }
 
@@ -411,14 +460,21 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
   g.ldy = swiglu ? w->N / 2 : w->N;
   g.out_f32 = out_dtype == SVDQ_OUT_F32 ? 1 : 0;
   g.epi = static_cast<int>(epi);
+  CUtensorMap tmY;
+  if (svdq_status s = make_tmap(&tmY, g.out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y,
+                                static_cast<uint64_t>(g.ldy), static_cast<uint64_t>(act->M),
+                                static_cast<uint64_t>(g.ldy) * (g.out_f32 ? 4 : 2), 32, 32,
+                                g.out_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+      s != SVDQ_OK)
+    return s;
   const int grid = g.num_tiles < sms ? g.num_tiles : sms;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (n_tile == 192) {
-    svdq::svdq_gemm_kernel<192, kStagesTile192><<<grid, 192, svdq::GemmLayout<192, kStagesTile192>::kSmem, st>>>(
-        tmA, tmB, tmU, tmL2, g);
+    svdq::svdq_gemm_kernel<192, kStagesTile192><<<grid, svdq::kGemmThreads, svdq::GemmLayout<192, kStagesTile192>::kSmem, st>>>(
+        tmA, tmB, tmU, tmL2, tmY, g);
   } else {
-    svdq::svdq_gemm_kernel<128, kStagesTile128><<<grid, 192, svdq::GemmLayout<128, kStagesTile128>::kSmem, st>>>(
-        tmA, tmB, tmU, tmL2, g);
+    svdq::svdq_gemm_kernel<128, kStagesTile128><<<grid, svdq::kGemmThreads, svdq::GemmLayout<128, kStagesTile128>::kSmem, st>>>(
+        tmA, tmB, tmU, tmL2, tmY, g);
   }
   return check_launch("svdq_gemm_kernel");
 }

@@ -13,12 +13,17 @@
 //               into a STAGES-deep shared-memory ring (full/empty mbarriers). Before a tile's K
 //               loop, ring slots carry the tile's U_hi, U_lo (128 x r) and L2^T (n_tile x r) in
 //               chunks of 32 columns of r.
-//   warp 1      TMEM allocator + single-thread MMA issuer: tcgen05.cp of the scale factors into
-//               TMEM, 4 x tcgen05.mma kind::mxf4nvf4 (M=128, N=n_tile, K=64) per K step, 2 r/16 x
+//   warp 1      TMEM allocator + single-thread MMA issuer:
+//               4 x tcgen05.mma kind::mxf4nvf4 (M=128, N=n_tile, K=64) per K step, 2 r/16 x
 //               kind::f16 (hi and lo halves of U against the same L2 tile) for the low-rank term; tcgen05.commit frees ring slots and publishes
 //               finished accumulators. Accumulators are double-buffered in TMEM when they fit.
 //   warps 2..5  epilogue: tcgen05.ld (each warp its 32-lane quadrant), y = alpha acc (+ bias),
 //               SwiGLU on interleaved gate/up columns, bf16 or fp32 store.
+//   warps 6..9  scale-factor writers: per K step, copy the stage's E4M3 scale atoms from shared
+//               memory into a double-buffered TMEM region with tcgen05.st (each warp its lane
+//               quadrant). Measured on B200, every tcgen05.cp costs ~64 tensor-pipe cycles whatever
+//               its shape, so copying 12 atoms per K step with tcgen05.cp starved the MMAs; stores
+//               from four warps run beside the MMAs without slowing them.
 // Every mbarrier wait is bounded (global timer); a wait that runs out records a status bit, sets
 // a shared abort flag so that the other roles stop too, and the kernel drains its own copies and
 // MMAs before freeing TMEM and returning.
@@ -55,15 +60,18 @@ struct GemmLayout {
   static constexpr int kOffB = kA;
   static constexpr int kOffSfa = kA + kB;
   static constexpr int kOffSfb = kA + kB + kSfa;
+  // TMEM scale-factor buffer (one K step): SFA 4 MMAs x 4 columns, then SFB 4 MMAs x 4 x atoms.
   static constexpr int kSfCols = 16 + 16 * kSfAtomsB;
-  static constexpr int kAccBufs = (2 * N_TILE + kSfCols <= 512) ? 2 : 1;
-  static constexpr int kColSfa = kAccBufs * N_TILE;
-  static constexpr int kColSfb = kColSfa + 16;
-  static constexpr int kBarOff = STAGES * kStage;
-  static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1;
+  static constexpr int kAccBufs = (2 * N_TILE + 2 * kSfCols <= 512) ? 2 : 1;
+  static constexpr int kColSf = kAccBufs * N_TILE;  // two buffers of kSfCols columns from here
+  // epilogue staging: 4 warps x 2 buffers x (32 rows x 32 columns of fp32 at most)
+  static constexpr int kStageOut = 32 * 32 * 4;
+  static constexpr int kOutOff = STAGES * kStage;
+  static constexpr int kBarOff = kOutOff + 4 * 2 * kStageOut;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1 + 4;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
-  static_assert(kColSfb + 16 * kSfAtomsB <= 512, "TMEM budget");
+  static_assert(kColSf + 2 * kSfCols <= 512, "TMEM budget");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -73,11 +81,22 @@ constexpr int kLrChunk = 32;
 constexpr int kOffULo = 128 * kLrChunk * 2;
 __device__ __forceinline__ uint32_t lr_swizzle_mode(int rc) { return rc == 16 ? 6u : 4u; }
 
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint4 (&v)[4]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0].x), "r"(v[0].y), "r"(v[0].z), "r"(v[0].w), "r"(v[1].x), "r"(v[1].y), "r"(v[1].z), "r"(v[1].w),
+      "r"(v[2].x), "r"(v[2].y), "r"(v[2].z), "r"(v[2].w), "r"(v[3].x), "r"(v[3].y), "r"(v[3].z), "r"(v[3].w)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+constexpr int kGemmThreads = 320;
+
 template <int N_TILE, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     svdq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
-                     const GemmArgs args) {
+                     const __grid_constant__ CUtensorMap tmY, const GemmArgs args) {
   using L = GemmLayout<N_TILE, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -88,6 +107,8 @@ __global__ void __launch_bounds__(192, 1)
   auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
   auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kAccBufs + b); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * L::kAccBufs);
+  auto sf_full_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * L::kAccBufs + 1 + b); };
+  auto sf_free_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * L::kAccBufs + 3 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -104,10 +125,15 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(acce_bar(b), 4);
     }
     mbar_init(drain_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sf_full_bar(b), 4);
+      mbar_init(sf_free_bar(b), 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmY);
     if (r > 0) {
       prefetch_tmap(&tmU);
       prefetch_tmap(&tmL2);
@@ -173,8 +199,8 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, acc = 0, sfb = 0;
+      uint32_t phase = 0, acc_phase = 0, sf_phase = 0;
       const uint32_t idesc_fp4 = idesc_nvfp4(128, N_TILE);
       const uint32_t idesc_lr = idesc_bf16(128, N_TILE);
       const int rc = r < kLrChunk ? r : kLrChunk;
@@ -205,24 +231,23 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
         for (int kt = 0; kt < args.k_iters; ++kt) {
           if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
+          // scale factors of this K step, written into TMEM buffer sfb by the scale-factor warps
+          if (!(ok = mbar_wait_bounded(sf_full_bar(sfb), sf_phase, wait_ns, status, kStatusMma, abort_flag))) break;
           tc_fence_after();
           const uint32_t sa = sbase + stage * L::kStage;
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tc_cp_sf(tmem + L::kColSfa + 4 * i, smem_desc(sa + L::kOffSfa + 512 * i, 0, 128, 0));
-#pragma unroll
-          for (int i = 0; i < 4 * L::kSfAtomsB; ++i)
-            tc_cp_sf(tmem + L::kColSfb + 4 * i, smem_desc(sa + L::kOffSfb + 512 * i, 0, 128, 0));
+          const uint32_t tsf = tmem + L::kColSf + sfb * L::kSfCols;
           const uint64_t da = smem_desc(sa, 16, 1024, 2);
           const uint64_t db = smem_desc(sa + L::kOffB, 16, 1024, 2);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            mma_nvfp4(d, da + 2u * i, db + 2u * i, idesc_fp4, tmem + L::kColSfa + 4 * i,
-                      tmem + L::kColSfb + 4 * L::kSfAtomsB * i, accumulate);
+            mma_nvfp4(d, da + 2u * i, db + 2u * i, idesc_fp4, tsf + 4 * i, tsf + 16 + 4 * L::kSfAtomsB * i,
+                      accumulate);
             accumulate = 1;
           }
           tc_commit(empty_bar(stage));
+          tc_commit(sf_free_bar(sfb));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++sfb == 2) { sfb = 0; sf_phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit(accf_bar(acc));
@@ -232,23 +257,101 @@ __global__ void __launch_bounds__(192, 1)
       tc_commit(drain_bar);
       mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
     }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------------ scale-factor writers (warps 6..9)
+    // Each warp owns one TMEM lane quadrant and writes into it the replicated scale-factor layout
+    // the block-scaled MMA reads: for a 128-row atom, lane l, column c holds the 4 E4M3 scales of
+    // row l + 32 c -- exactly bytes [16 l, 16 l + 16) of the 512-byte atom in shared memory.
+    const int q = warp & 3;
+    int stage = 0, sfb = 0;
+    uint32_t phase = 0, sf_phase = 0;
+    const int lr_slots = (r + kLrChunk - 1) / kLrChunk;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+      for (int c = 0; c < lr_slots; ++c)
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      for (int kt = 0; kt < args.k_iters; ++kt) {
+        bool got = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
+        got = got && mbar_wait_bounded(sf_free_bar(sfb), sf_phase ^ 1u, wait_ns, status, kStatusEpilogue, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        const uint8_t* sfs = smem + stage * L::kStage + L::kOffSfa + lane * 16;
+        const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kColSf + sfb * L::kSfCols;
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
+        tmem_st_x16(tsf, v);
+#pragma unroll
+        for (int h = 0; h < L::kSfAtomsB; ++h) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            v[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + L::kOffSfb + lane * 16 + 512 * (4 * h + i));
+          tmem_st_x16(tsf + 16 + 16 * h, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_full_bar(sfb));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++sfb == 2) { sfb = 0; sf_phase ^= 1u; }
+      }
+    }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
+    // Each warp drains its 32-lane TMEM quadrant 32 columns at a time, applies alpha / bias /
+    // SwiGLU, writes the 32 x 32 block into a swizzled shared-memory buffer (64B swizzle for bf16,
+    // 128B for fp32 rows: conflict-free 16-byte writes) and one lane stores it with a TMA tensor
+    // store; two buffers per warp let the next block fill while the previous store drains. Rows at
+    // or beyond M are clipped by the tensor map.
     const int q = warp & 3;
     const float alpha = *args.alpha;
     const bool has_bias = (args.epi & 1) != 0;
     const bool swiglu = (args.epi & 2) != 0;
+    const bool f32 = args.out_f32 != 0;
     const int hN = args.N >> 1;
+    uint8_t* stage_out = smem + L::kOutOff + q * 2 * L::kStageOut;
+    int buf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
+    auto emit = [&](const float (&v)[32], int row0, int col0) {
+      // buffer reuse: the store issued from it two blocks ago has finished reading
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+      uint8_t* dst = stage_out + buf * L::kStageOut;
+      if (f32) {
+        // 128-byte rows, 8 chunks of 16 bytes; chunk j of row `lane` lives at j ^ (lane % 8)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(dst + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+              make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      } else {
+        // 64-byte rows, 4 chunks; chunk j of row `lane` lives at j ^ ((lane / 2) % 4)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+            w[e] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(dst + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tmY, smem_addr(dst), col0, row0);
+        bulk_commit_group();
+      }
+      buf ^= 1;
+    };
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
       const int m_blk = tile % args.m_tiles, n_blk = tile / args.m_tiles;
       // warp-uniform outcome: tcgen05.ld below is a .sync.aligned warp instruction
       const bool got = mbar_wait_bounded(accf_bar(acc), acc_phase, wait_ns, status, kStatusEpilogue, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const int row = m_blk * 128 + q * 32 + lane;
-      const bool row_ok = row < args.M;
+      const int row0 = m_blk * 128 + q * 32;
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * N_TILE);
       if (!swiglu) {
 #pragma unroll 1
@@ -256,6 +359,12 @@ __global__ void __launch_bounds__(192, 1)
           float v[32];
           tmem_ld_32x32(tb + c * 32, v);
           tmem_wait_ld();
+          if (c == N_TILE / 32 - 1) {
+            // all of this accumulator is in registers or already consumed: hand it back early
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce_bar(acc));
+          }
           const int n0 = n_blk * N_TILE + c * 32;
           if (has_bias) {
 #pragma unroll
@@ -269,25 +378,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = alpha * v[i];
           }
-          if (row_ok) {
-            if (args.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + static_cast<size_t>(row) * args.ldy + n0);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + static_cast<size_t>(row) * args.ldy + n0);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint32_t w[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
-                  w[j] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            }
-          }
+          emit(v, row0, n0);
         }
       } else {
         constexpr int kHalf = N_TILE / 2;
@@ -297,6 +388,11 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld_32x32(tb + c * 32, gt);
           tmem_ld_32x32(tb + kHalf + c * 32, up);
           tmem_wait_ld();
+          if (c == kHalf / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce_bar(acc));
+          }
           const int j0 = n_blk * kHalf + c * 32;
           if (has_bias) {
 #pragma unroll
@@ -319,32 +415,14 @@ __global__ void __launch_bounds__(192, 1)
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i) gt[i] = gt[i] / (1.0f + __expf(-gt[i])) * up[i];
-          if (row_ok) {
-            if (args.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + static_cast<size_t>(row) * args.ldy + j0);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) dst[i] = make_float4(gt[4 * i], gt[4 * i + 1], gt[4 * i + 2], gt[4 * i + 3]);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + static_cast<size_t>(row) * args.ldy + j0);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint32_t w[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const __nv_bfloat162 h = __floats2bfloat162_rn(gt[8 * i + 2 * j], gt[8 * i + 2 * j + 1]);
-                  w[j] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            }
-          }
+          emit(gt, row0, j0);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar(acc));
       if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
+    // every TMA store issued by this warp has completed before the CTA may exit
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -88,133 +88,292 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA in the cluster arrives (warp-converged: .aligned).
+__device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // ------------------------------------------------------------------------------------------------
 // Kernel 1: smoothing + NVFP4 activation quantization + U = X L1s, one pass over X.
-// U is stored divided by alpha = g_x g_w (so the GEMM applies one scale at the end) as a bf16
-// hi/lo pair.
-// CTA = 16 rows x all of K, 8 warps splitting K in 32-column chunks. Within a warp, lane (g, t)
-// (g = lane/4, t = lane%4) loads 8 consecutive bf16 of rows g and g+8 with 128-bit loads; the same
-// registers are both the quantizer's input and the A fragments of two m16n8k16 bf16 MMAs (the
-// reduction index is permuted consistently in A and B, which leaves the product unchanged).
+//
+// A CTA owns 128 rows of X and a K range (a cluster of 1, 2 or 4 CTAs splits K when there are few
+// row tiles). TMA streams 128 x 64 bf16 stages (128B swizzle) of X, and 64-column slices of
+// L1s^T, into a 4-deep shared-memory ring. Every stage is read twice from shared memory: by eight
+// quantizer warps (smoothing, block amax, E4M3 scale, E2M1 codes; codes and scales go straight to
+// global memory), and by a single-thread tcgen05 bf16 MMA (M=128, N=r, K=16) that accumulates the
+// down-projection in TMEM. X thus crosses HBM once. At the end four warps read U from TMEM; with
+// a K split the partial U of every CTA is summed in rank order through distributed shared memory.
+// U is stored divided by alpha = g_x g_w (one scale for the whole GEMM) as a bf16 hi/lo pair.
+constexpr int kQThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 quantize (2..5 also drain U)
+constexpr int kQStages = 4;
+constexpr int kQTile = 128 * 128;  // 128 rows x 64 bf16
+
+template <int R>
+struct QuantLayout {
+  static constexpr int kL1 = (R * 128 + 1023) / 1024 * 1024;
+  static constexpr int kStage = kQTile + kL1;
+  static constexpr int kPartOff = kQStages * kStage;
+  static constexpr int kPart = R * 128 * 4 + 128 * 4;  // rows padded to R + 1 floats
+  static constexpr int kBarOff = kPartOff + kPart;
+  static constexpr int kNumBars = 2 * kQStages + 2;
+  static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
+  static constexpr int kTmemCols = R <= 32 ? 32 : 64;
+  static_assert(kStage % 1024 == 0, "stage alignment");
+};
+
 struct QuantActArgs {
-  const __nv_bfloat16* X;
   const float* inv_lambda;
-  const __nv_bfloat16* L1s_t;  // [r][K]
   const float* g_x;
   const float* g_w;
   uint8_t* codes;              // [M_pad][K/2]
   uint8_t* sf;                 // activation MMA layout
   __nv_bfloat16* U;            // [2][M_pad][r]: hi then lo
   float* alpha;
-  int M, K, M_pad;
+  unsigned long long wait_ns;
+  int M, K, M_pad, k_per_cta;
 };
 
 template <int R>
-__global__ void __launch_bounds__(256) quant_act_kernel(const QuantActArgs a) {
-  constexpr int NT = R / 8;
-  __shared__ float part[R > 0 ? 8 * 16 * R : 1];
+__global__ void __launch_bounds__(kQThreads, 2)
+    quant_act_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL1,
+                     const QuantActArgs a) {
+  using L = QuantLayout<R>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kQStages + s); };
+  const uint32_t accf_bar = bar0 + 8u * (2 * kQStages);
+  const uint32_t drain_bar = accf_bar + 8u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int m0 = blockIdx.x * 16;
-  const int rowA = m0 + g, rowB = m0 + g + 8;
-  const bool okA = rowA < a.M, okB = rowB < a.M;
+  const uint32_t csize = cluster_nctarank(), crank = cluster_ctarank();
+  const int m_tile = blockIdx.x / csize;
+  const int kbeg = static_cast<int>(crank) * a.k_per_cta;
+  const int n_steps = a.k_per_cta >> 6;
   const int K = a.K;
-  const float gx = *a.g_x;
-  const float d6 = __fmul_rn(6.0f, gx);
-  const __nv_bfloat16* xA = a.X + static_cast<size_t>(okA ? rowA : 0) * K;
-  const __nv_bfloat16* xB = a.X + static_cast<size_t>(okB ? rowB : 0) * K;
-  uint8_t* cA = a.codes + static_cast<size_t>(rowA) * (K >> 1);
-  uint8_t* cB = a.codes + static_cast<size_t>(rowB) * (K >> 1);
+  unsigned* status = &g_svdq_status;
+  const uint64_t wait_ns = a.wait_ns;
 
-  float acc[NT > 0 ? NT : 1][4];
-#pragma unroll
-  for (int j = 0; j < (NT > 0 ? NT : 1); ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-
-  const int nchunks = K >> 5;
-  const uint4 zero = make_uint4(0, 0, 0, 0);
-  int c = warp;
-  uint4 xa = zero, xb = zero;
-  if (c < nchunks) {
-    const int k = (c << 5) + (t << 3);
-    if (okA) xa = ldg_stream(xA + k);
-    if (okB) xb = ldg_stream(xB + k);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 8 + (R > 0 ? 1 : 0));
+    }
+    mbar_init(accf_bar, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmX);
+    if (R > 0) prefetch_tmap(&tmL1);
   }
-  for (; c < nchunks; c += 8) {
-    const int k = (c << 5) + (t << 3);
-    // prefetch the next chunk of this warp before working on the current one
-    uint4 na = zero, nb = zero;
-    if (c + 8 < nchunks) {
-      if (okA) na = ldg_stream(xA + k + 256);
-      if (okB) nb = ldg_stream(xB + k + 256);
+  if (R > 0 && warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = R > 0 ? *tmem_slot : 0u;
+  const float gx = *a.g_x;
+  const float alpha = __fmul_rn(gx, *a.g_w);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
+      for (int st = 0; st < n_steps; ++st) {
+        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)) break;
+        const uint32_t sa = sbase + stage * L::kStage;
+        mbar_arrive_expect_tx(full_bar(stage), kQTile + R * 128);
+        const int kx = kbeg + (st << 6);
+        tma_load_2d(sa, &tmX, kx, m_tile * 128, full_bar(stage));
+        if (R > 0) tma_load_2d(sa + kQTile, &tmL1, kx, 0, full_bar(stage));
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+      }
+      for (int s = 0; s < kQStages; ++s)
+        if (armed & (1u << s))
+          mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
     }
-    const float4 l0 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k));
-    const float4 l1 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k + 4));
-    const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-    float va[8], vb[8];
-    bf16x8_to_f32(xa, va);
-    bf16x8_to_f32(xb, vb);
+  } else if (warp == 1) {
+    if (R > 0 && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, accumulate = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_bf16(128, R);
+      for (int st = 0; st < n_steps; ++st) {
+        if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t sa = sbase + stage * L::kStage;
+        const uint64_t dx = smem_desc(sa, 16, 1024, 2);
+        const uint64_t dl = smem_desc(sa + kQTile, 16, 1024, 2);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      va[i] = __fmul_rn(va[i], lam[i]);
-      vb[i] = __fmul_rn(vb[i], lam[i]);
+        for (int j = 0; j < 4; ++j) {
+          mma_bf16(tmem, dx + 2u * j, dl + 2u * j, idesc, accumulate);
+          accumulate = 1;
+        }
+        tc_commit(empty_bar(stage));
+        if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+      }
+      if (ok) tc_commit(accf_bar);
+      tc_commit(drain_bar);
+      mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
     }
-    uint32_t sa, sb;
-    const uint32_t qa = nvfp4_half_block(va, gx, d6, sa);
-    const uint32_t qb = nvfp4_half_block(vb, gx, d6, sb);
-    *reinterpret_cast<uint32_t*>(cA + (k >> 1)) = qa;
-    *reinterpret_cast<uint32_t*>(cB + (k >> 1)) = qb;
-    if ((t & 1) == 0) {
-      a.sf[act_sf_offset(rowA, k >> 4, K)] = static_cast<uint8_t>(sa);
-      a.sf[act_sf_offset(rowB, k >> 4, K)] = static_cast<uint8_t>(sb);
+  } else {
+    // quantizers: warp w (0..7) handles rows 4w + lane/8 + 32i (i = 0..3), chunk lane%8 of 8 bf16;
+    // the lanes of one row read its 128 swizzled bytes in one conflict-free 128-byte phase.
+    const int w = warp - 2;
+    const int c = lane & 7;
+    const float d6 = __fmul_rn(6.0f, gx);
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int st = 0; st < n_steps; ++st) {
+      const bool got = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const int k = kbeg + (st << 6) + (c << 3);
+      const float4 l0 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k));
+      const float4 l1 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k + 4));
+      const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+      const uint8_t* tile = smem + stage * L::kStage;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rl = 4 * w + (lane >> 3) + 32 * i;
+        const uint4 x = *reinterpret_cast<const uint4*>(tile + rl * 128 + ((c ^ (rl & 7)) << 4));
+        float v[8];
+        bf16x8_to_f32(x, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], lam[e]);
+        uint32_t sc;
+        const uint32_t q = nvfp4_half_block(v, gx, d6, sc);
+        const int row = m_tile * 128 + rl;
+        *reinterpret_cast<uint32_t*>(a.codes + static_cast<size_t>(row) * (K >> 1) + (k >> 1)) = q;
+        // the row's four block scales (chunks 0, 2, 4, 6) form one 32-bit word of the scale atom
+        const int base = lane & ~7;
+        const uint32_t s0 = __shfl_sync(0xffffffffu, sc, base);
+        const uint32_t s1 = __shfl_sync(0xffffffffu, sc, base + 2);
+        const uint32_t s2 = __shfl_sync(0xffffffffu, sc, base + 4);
+        const uint32_t s3 = __shfl_sync(0xffffffffu, sc, base + 6);
+        if (c == 0)
+          *reinterpret_cast<uint32_t*>(a.sf + act_sf_offset(row, (kbeg + (st << 6)) >> 4, K)) =
+              s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(stage));
+      if (++stage == kQStages) { stage = 0; phase ^= 1u; }
     }
     if constexpr (R > 0) {
+      // warps 2..5 (quadrant q = warp % 4) read this CTA's rows of U from TMEM; a lone CTA
+      // finishes them at once, a cluster member parks its partial in shared memory for the
+      // cluster's first CTA, which adds the partials in rank order.
+      const int q = warp & 3;
+      const bool mine_rows = warp < 6;
+      bool got = true;
+      if (mine_rows) got = mbar_wait_bounded(accf_bar, 0, wait_ns, status, kStatusEpilogue, abort_flag);
+      got = __all_sync(0xffffffffu, got) && mine_rows;
+      float u[R];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const uint4 bq = __ldg(reinterpret_cast<const uint4*>(a.L1s_t + static_cast<size_t>(j * 8 + g) * K + k));
-        mma_bf16_16816(acc[j], xa.x, xb.x, xa.y, xb.y, bq.x, bq.y);
-        mma_bf16_16816(acc[j], xa.z, xb.z, xa.w, xb.w, bq.z, bq.w);
+      for (int j = 0; j < R; ++j) u[j] = 0.0f;
+      if (got) {
+        tc_fence_after();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        if constexpr (R == 16) {
+          uint32_t rr[16];
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+              : "=r"(rr[0]), "=r"(rr[1]), "=r"(rr[2]), "=r"(rr[3]), "=r"(rr[4]), "=r"(rr[5]), "=r"(rr[6]), "=r"(rr[7]),
+                "=r"(rr[8]), "=r"(rr[9]), "=r"(rr[10]), "=r"(rr[11]), "=r"(rr[12]), "=r"(rr[13]), "=r"(rr[14]),
+                "=r"(rr[15])
+              : "r"(ta));
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) u[e] = __uint_as_float(rr[e]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < R; j += 32) {
+            float t[32];
+            tmem_ld_32x32(ta + j, t);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[j + e] = t[e];
+          }
+        }
+        if (csize > 1 && crank != 0) {
+          float* part = reinterpret_cast<float*>(smem + L::kPartOff) + (q * 32 + lane) * (R + 1);
+#pragma unroll
+          for (int j = 0; j < R; ++j) part[j] = u[j];
+        }
+      }
+      if (csize > 1) cluster_sync_all();
+      if (got && crank == 0) {
+        const int rl = q * 32 + lane;
+        for (uint32_t rk = 1; rk < csize; ++rk) {
+          const uint32_t pa = cluster_map(smem_addr(smem + L::kPartOff) + rl * (R + 1) * 4, rk);
+#pragma unroll
+          for (int j = 0; j < R; ++j) u[j] += ld_cluster_f32(pa + j * 4);
+        }
+        const float cinv = __frcp_rn(alpha);
+        __nv_bfloat16* u_hi = a.U + (static_cast<size_t>(m_tile) * 128 + rl) * R;
+        __nv_bfloat16* u_lo = u_hi + static_cast<size_t>(a.M_pad) * R;
+#pragma unroll
+        for (int j = 0; j < R; j += 8) {
+          uint32_t wh[4], wl[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float v0 = __fmul_rn(u[j + 2 * e], cinv), v1 = __fmul_rn(u[j + 2 * e + 1], cinv);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(v0, v1);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(__fsub_rn(v0, __low2float(hi)), __fsub_rn(v1, __high2float(hi)));
+            wh[e] = *reinterpret_cast<const uint32_t*>(&hi);
+            wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
+          }
+          *reinterpret_cast<uint4*>(u_hi + j) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          *reinterpret_cast<uint4*>(u_lo + j) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
       }
     }
-    xa = na;
-    xb = nb;
   }
 
-  const float alpha = __fmul_rn(gx, *a.g_w);
-  if constexpr (R > 0) {
-    float* pw = part + warp * 16 * R;
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int col = j * 8 + 2 * t;
-      pw[g * R + col] = acc[j][0];
-      pw[g * R + col + 1] = acc[j][1];
-      pw[(g + 8) * R + col] = acc[j][2];
-      pw[(g + 8) * R + col + 1] = acc[j][3];
-    }
-    __syncthreads();
-    // U / alpha as a bf16 pair: hi = bf16(u), lo = bf16(u - hi) (the difference is exact in fp32),
-    // so that two bf16 MMAs against L2 carry about 16 significant bits of the branch.
-    const float cinv = __frcp_rn(alpha);
-    __nv_bfloat16* u_hi = a.U + static_cast<size_t>(m0) * R;
-    __nv_bfloat16* u_lo = u_hi + static_cast<size_t>(a.M_pad) * R;
-    for (int i = threadIdx.x; i < 16 * R; i += 256) {
-      float s = 0.0f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) s += part[w * 16 * R + i];
-      const float u = __fmul_rn(s, cinv);
-      const __nv_bfloat16 hi = __float2bfloat16_rn(u);
-      u_hi[i] = hi;
-      u_lo[i] = __float2bfloat16_rn(__fsub_rn(u, __bfloat162float(hi)));
-    }
+  if constexpr (R == 0) {
+    if (csize > 1) cluster_sync_all();
+  } else {
+    // warps 0 and 1 take part in the cluster barrier the quantizer warps passed above
+    if (csize > 1 && warp < 2) cluster_sync_all();
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.alpha = alpha;
+  // peers keep their shared memory until the leader has read it
+  if (csize > 1) cluster_sync_all();
+  tc_fence_before();
+  __syncthreads();
+  if (R > 0 && warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
