@@ -88,6 +88,15 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
+// Two IEEE round-to-nearest fp32 products in one instruction (lane-wise, same rounding as __fmul_rn).
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&r);
+}
+
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -136,7 +145,8 @@ struct QuantLayout {
   static constexpr int kStage = kQTile + kL1;
   static constexpr int kPartOff = kQStages * kStage;
   static constexpr int kPart = R * 128 * 4 + 128 * 4;  // rows padded to R + 1 floats
-  static constexpr int kBarOff = kPartOff + kPart;
+  static constexpr int kTabOff = kPartOff + kPart;        // 128 fp32: 1 / (dec(s) g_x) per scale code
+  static constexpr int kBarOff = kTabOff + 128 * 4;
   static constexpr int kNumBars = 2 * kQStages + 2;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
   static constexpr int kTmemCols = R <= 32 ? 32 : 64;
@@ -199,9 +209,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = R > 0 ? *tmem_slot : 0u;
   const float gx = *a.g_x;
   const float alpha = __fmul_rn(gx, *a.g_w);
+  float* rs_tab = reinterpret_cast<float*>(smem + L::kTabOff);
+  if (threadIdx.x < 128) rs_tab[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_value(threadIdx.x), gx));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = R > 0 ? *tmem_slot : 0u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -247,42 +262,70 @@ __global__ void __launch_bounds__(kQThreads, 2)
       mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
     }
   } else {
-    // quantizers: warp w (0..7) handles rows 4w + lane/8 + 32i (i = 0..3), chunk lane%8 of 8 bf16;
-    // the lanes of one row read its 128 swizzled bytes in one conflict-free 128-byte phase.
-    const int w = warp - 2;
-    const int c = lane & 7;
+    // quantizers: thread t of the 256 owns 16-element block b = t % 4 of rows t / 4 and t / 4 + 64
+    // of the stage. The four threads of a row read its 128 swizzled bytes; a warp's 16-byte reads
+    // cover 8 rows x 4 blocks and stay conflict-free (chunks 2b and 2b+1 XOR row % 8).
+    const int t = threadIdx.x - 64;
+    const int b = t & 3;
     const float d6 = __fmul_rn(6.0f, gx);
     int stage = 0;
     uint32_t phase = 0;
     for (int st = 0; st < n_steps; ++st) {
       const bool got = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
-      const int k = kbeg + (st << 6) + (c << 3);
-      const float4 l0 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k));
-      const float4 l1 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k + 4));
-      const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+      const int kst = kbeg + (st << 6);
+      const int k = kst + (b << 4);
+      float2 lam[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 l = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k) + j);
+        lam[2 * j] = make_float2(l.x, l.y);
+        lam[2 * j + 1] = make_float2(l.z, l.w);
+      }
       const uint8_t* tile = smem + stage * L::kStage;
+      uint4 x[2][2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int rl = 4 * w + (lane >> 3) + 32 * i;
-        const uint4 x = *reinterpret_cast<const uint4*>(tile + rl * 128 + ((c ^ (rl & 7)) << 4));
-        float v[8];
-        bf16x8_to_f32(x, v);
+      for (int i = 0; i < 2; ++i) {
+        const int rl = (t >> 2) + 64 * i;
+        x[i][0] = *reinterpret_cast<const uint4*>(tile + rl * 128 + (((2 * b) ^ (rl & 7)) << 4));
+        x[i][1] = *reinterpret_cast<const uint4*>(tile + rl * 128 + (((2 * b + 1) ^ (rl & 7)) << 4));
+      }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], lam[e]);
-        uint32_t sc;
-        const uint32_t q = nvfp4_half_block(v, gx, d6, sc);
+      for (int i = 0; i < 2; ++i) {
+        const int rl = (t >> 2) + 64 * i;
+        const uint32_t wx[8] = {x[i][0].x, x[i][0].y, x[i][0].z, x[i][0].w, x[i][1].x, x[i][1].y, x[i][1].z, x[i][1].w};
+        float2 v[8];
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[j] = mul2_rn(make_float2(__uint_as_float(wx[j] << 16), __uint_as_float(wx[j] & 0xFFFF0000u)), lam[j]);
+          amax = fmaxf(amax, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
+        }
+        const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, d6));
+        uint2 codes = make_uint2(0u, 0u);
+        if (sc != 0) {
+          const float r = rs_tab[sc];
+          const float2 r2 = make_float2(r, r);
+          float q[16];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float2 p = mul2_rn(v[j], r2);
+            q[2 * j] = p.x;
+            q[2 * j + 1] = p.y;
+          }
+          codes.x = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q));
+          codes.y = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q + 8));
+        }
         const int row = m_tile * 128 + rl;
-        *reinterpret_cast<uint32_t*>(a.codes + static_cast<size_t>(row) * (K >> 1) + (k >> 1)) = q;
-        // the row's four block scales (chunks 0, 2, 4, 6) form one 32-bit word of the scale atom
-        const int base = lane & ~7;
+        *reinterpret_cast<uint2*>(a.codes + static_cast<size_t>(row) * (K >> 1) + (k >> 1)) = codes;
+        // the row's four block scales form one 32-bit word of the scale atom
+        const int base = (threadIdx.x & 31) & ~3;
         const uint32_t s0 = __shfl_sync(0xffffffffu, sc, base);
-        const uint32_t s1 = __shfl_sync(0xffffffffu, sc, base + 2);
-        const uint32_t s2 = __shfl_sync(0xffffffffu, sc, base + 4);
-        const uint32_t s3 = __shfl_sync(0xffffffffu, sc, base + 6);
-        if (c == 0)
-          *reinterpret_cast<uint32_t*>(a.sf + act_sf_offset(row, (kbeg + (st << 6)) >> 4, K)) =
-              s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        const uint32_t s1 = __shfl_sync(0xffffffffu, sc, base + 1);
+        const uint32_t s2 = __shfl_sync(0xffffffffu, sc, base + 2);
+        const uint32_t s3 = __shfl_sync(0xffffffffu, sc, base + 3);
+        if (b == 0)
+          *reinterpret_cast<uint32_t*>(a.sf + act_sf_offset(row, kst >> 4, K)) = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(stage));
