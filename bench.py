@@ -32,6 +32,10 @@ METRIC = "W4A4+low-rank linear TFLOPS, % of B200 dense FP4 peak; tokens/s per la
 DEFAULT_WORKLOAD = "qkv_2048"
 FP4_PER_BF16 = 4.0   # nominal dense FP4 / dense bf16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
 FLUSH_BYTES = 256 << 20
+# DRAM bytes (read + write) per launch of the GEMM, from the ncu capture summarised in
+# profiles/svdq_gemm_kernel_qkv2048.md, keyed by a hash of the kernel source it was taken on; any
+# change to the kernel source makes the figure stale and it is reported as null.
+PROFILED_GEMM_TRAFFIC = {("qkv_2048", "bca0a427a7ee"): 350.05e6}
 
 
 def read_peaks():
@@ -96,13 +100,31 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def gemm_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("svdq_gemm.cuh", "svdq_ptx.cuh"):
+        with open(os.path.join(ROOT, "bit_diffusion_transformer_svdquant_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Largest value over all ranks (the slowest replica sets the time)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def layer_flops(spec):
     return 2.0 * spec.M * spec.N * spec.K, 2.0 * spec.M * spec.r * (spec.K + spec.N)
 
 
 def kernel1_bytes(spec):
-    """Algorithmic HBM bytes of kernel 1: read X (bf16), write codes + scales + U (bf16)."""
-    return spec.M * spec.K * 2 + spec.M * spec.K // 2 + spec.M * spec.K // 16 + spec.M * spec.r * 2
+    """Algorithmic HBM bytes of kernel 1: read X (bf16), write codes + scales + U (bf16 hi and lo)."""
+    return spec.M * spec.K * 2 + spec.M * spec.K // 2 + spec.M * spec.K // 16 + spec.M * spec.r * 4
 
 
 # ---------------------------------------------------------------------------------------------- GPU arm
@@ -192,10 +214,7 @@ def gpu_arm(args, rank, world, dev):
     total_ms = float(sum(step_ms))
     k1_ms = [[k_ev[s][i][0].elapsed_time(k_ev[s][i][1]) for s in range(K)] for i in range(n_l)]
     k2_ms = [[k_ev[s][i][1].elapsed_time(k_ev[s][i][2]) for s in range(K)] for i in range(n_l)]
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     flops_main = sum(layer_flops(L["spec"])[0] for L in layers)
     flops_lr = sum(layer_flops(L["spec"])[1] for L in layers)
@@ -237,7 +256,8 @@ def gpu_arm(args, rank, world, dev):
         },
         "roofline": {"bound": "tensor", "kernel": "svdq_gemm_kernel", "achieved": round(achieved, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
-                     "traffic": None,
+                     "traffic": PROFILED_GEMM_TRAFFIC.get((wl.name, gemm_source_hash())),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_PER_BF16}"
                                     " (nominal dense FP4/bf16 ratio)",
                      "algorithmic": f"{gemm_flops / 1e9:.1f} GFLOP per launch (2MNK + 2MrN)"},
@@ -303,12 +323,18 @@ def oracle_step(prepared, rows):
 
 
 def choose_rows(prepared, target_s):
-    rows = 64
-    t0 = time.perf_counter()
-    oracle_step(prepared, rows)
-    dt = time.perf_counter() - t0
+    """Rows of the workload whose oracle forward takes about target_s on this host (the per-call
+    weight decode is a fixed cost, so the time is fitted as a + b * rows from two trials)."""
     M = prepared[0]["spec"].M
-    return int(max(16, min(M, rows * target_s / max(dt, 1e-3))))
+    oracle_step(prepared, 32)  # warm caches and BLAS threads
+    ts = []
+    for rows in (64, 256):
+        t0 = time.perf_counter()
+        oracle_step(prepared, rows)
+        ts.append(time.perf_counter() - t0)
+    b = max((ts[1] - ts[0]) / 192.0, 1e-6)
+    a = max(ts[0] - 64 * b, 0.0)
+    return int(max(16, min(M, (target_s - a) / b)))
 
 
 def cpu_cores():
@@ -363,7 +389,7 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])

@@ -71,3 +71,33 @@ def test_no_gpu_fails_loudly(L):
     p = ctypes.c_void_p(1 << 40)
     st = L.svdq_pack_weight(p, p, p, p, 512, 512, 16, 0, p, 1 << 30, ctypes.byref(w), None)
     assert st == 3, (st, L.svdq_last_error())
+
+
+def _rank_main(rank, world, port, q):
+    import os
+    import torch
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    got = bench.max_over_ranks(1.5 + rank, torch.device("cpu"))
+    torch.distributed.barrier()
+    torch.distributed.destroy_process_group()
+    q.put((rank, got))
+
+
+def test_bench_max_over_ranks_gloo():
+    """The N>1 bench path (replicas): the reported time is the slowest rank's, on a 2-rank gloo group."""
+    import multiprocessing as mp
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert res == {0: 2.5, 1: 2.5}
