@@ -198,62 +198,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    // Measured on B200: the tensor pipe takes one tcgen05 instruction at a time (>= 64 cycles each,
+    // N/2 cycles for an NVFP4 MMA), and the next MMA issue returns only when the previous MMA is done,
+    // so the issuing thread's other work overlaps only the one MMA in flight. Per K step it therefore
+    // does one commit (which also frees the step's scale buffer: the writers watch the stage release)
+    // and waits for the next step's scales between the third and fourth MMA. A K step waits only on
+    // its scale buffer: the writers arrive there after they have seen the stage's data land.
     if (lane == 0) {
-      int stage = 0, acc = 0, sfb = 0;
-      uint32_t phase = 0, acc_phase = 0, sf_phase = 0;
+      const int num_tiles = args.num_tiles, k_iters = args.k_iters;
+      const int rc = r < kLrChunk ? r : kLrChunk;
+      const int nj = rc >> 4;
       const uint32_t idesc_fp4 = idesc_nvfp4(128, N_TILE);
       const uint32_t idesc_lr = idesc_bf16(128, N_TILE);
-      const int rc = r < kLrChunk ? r : kLrChunk;
-      const uint32_t lr_swz = lr_swizzle_mode(rc);
-      const uint32_t lr_sbo = 8u * rc * 2u;
+      // descriptor halves: low = start address / 16 | LBO (16 B) / 16 << 16; high = SBO / 16 |
+      // version 1 | swizzle mode << 29
+      const uint32_t lo0 = (sbase >> 4) | (1u << 16);
+      const uint32_t hi_ab = (1024u >> 4) | (1u << 14) | (2u << 29);
+      const uint32_t hi_lr = ((8u * rc * 2u) >> 4) | (1u << 14) | (lr_swizzle_mode(rc) << 29);
+      const uint32_t tsf0 = tmem + L::kColSf;
+      int stage = 0, sfb = 0, acc = 0;
+      uint32_t phase = 0, sf_phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-        if (!(ok = mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, wait_ns, status, kStatusMma, abort_flag)))
-          break;
-        tc_fence_after();
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        if (!(ok = mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, wait_ns, status, kStatusMma, abort_flag))) break;
         const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
         uint32_t accumulate = 0;
         for (int c0 = 0; c0 < r; c0 += kLrChunk) {
           if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
           tc_fence_after();
-          const uint32_t sa = sbase + stage * L::kStage;
-          const uint64_t dhi = smem_desc(sa, 16, lr_sbo, lr_swz);
-          const uint64_t dlo = smem_desc(sa + kOffULo, 16, lr_sbo, lr_swz);
-          const uint64_t dl = smem_desc(sa + L::kOffB, 16, lr_sbo, lr_swz);
-          for (int j = 0; j < (rc >> 4); ++j) {
-            mma_bf16(d, dhi + 2u * j, dl + 2u * j, idesc_lr, accumulate);
-            mma_bf16(d, dlo + 2u * j, dl + 2u * j, idesc_lr, 1u);
+          const uint32_t lo = lo0 + stage * (L::kStage >> 4);
+          for (int j = 0; j < nj; ++j) {
+            mma_bf16(d, desc_join(lo + 2u * j, hi_lr), desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr), idesc_lr,
+                     accumulate);
+            mma_bf16(d, desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr), desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr),
+                     idesc_lr, 1u);
             accumulate = 1;
           }
           tc_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        for (int kt = 0; kt < args.k_iters; ++kt) {
-          if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
-          // scale factors of this K step, written into TMEM buffer sfb by the scale-factor warps
-          if (!(ok = mbar_wait_bounded(sf_full_bar(sfb), sf_phase, wait_ns, status, kStatusMma, abort_flag))) break;
+        // the tile's first K step: its scales
+        if (!(ok = mbar_wait_bounded(sf_full_bar(sfb), sf_phase, wait_ns, status, kStatusMma, abort_flag))) break;
+        tc_fence_after();
+        for (int kt = 0; kt < k_iters; ++kt) {
+          const uint32_t la = lo0 + stage * (L::kStage >> 4);
+          const uint32_t lb = la + (L::kOffB >> 4);
+          const uint32_t tsf = tsf0 + sfb * L::kSfCols;
+          mma_nvfp4(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_fp4, tsf, tsf + 16, accumulate);
+          mma_nvfp4(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_fp4, tsf + 4,
+                    tsf + 16 + 4 * L::kSfAtomsB, 1u);
+          mma_nvfp4(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_fp4, tsf + 8,
+                    tsf + 16 + 8 * L::kSfAtomsB, 1u);
+          accumulate = 1;
+          const int nsfb = sfb ^ 1;
+          const uint32_t nsf_phase = sf_phase ^ static_cast<uint32_t>(sfb);
+          if (kt + 1 < k_iters)
+            ok = mbar_wait_bounded(sf_full_bar(nsfb), nsf_phase, wait_ns, status, kStatusMma, abort_flag);
           tc_fence_after();
-          const uint32_t sa = sbase + stage * L::kStage;
-          const uint32_t tsf = tmem + L::kColSf + sfb * L::kSfCols;
-          const uint64_t da = smem_desc(sa, 16, 1024, 2);
-          const uint64_t db = smem_desc(sa + L::kOffB, 16, 1024, 2);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            mma_nvfp4(d, da + 2u * i, db + 2u * i, idesc_fp4, tsf + 4 * i, tsf + 16 + 4 * L::kSfAtomsB * i,
-                      accumulate);
-            accumulate = 1;
-          }
+          mma_nvfp4(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_fp4, tsf + 12,
+                    tsf + 16 + 12 * L::kSfAtomsB, 1u);
           tc_commit(empty_bar(stage));
-          tc_commit(sf_free_bar(sfb));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++sfb == 2) { sfb = 0; sf_phase ^= 1u; }
+          sfb = nsfb;
+          sf_phase = nsf_phase;
+          if (!ok) break;
         }
         if (!ok) break;
         tc_commit(accf_bar(acc));
         if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
-      // Drain: all issued MMAs and scale copies complete before TMEM is freed.
+      // Drain: all issued MMAs complete before TMEM is freed.
       tc_commit(drain_bar);
       mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
     }
@@ -265,33 +280,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     int stage = 0, sfb = 0;
     uint32_t phase = 0, sf_phase = 0;
+    // (stage, phase) of the last two K steps: buffer sfb was last read by the K step two back, and
+    // the MMA thread's release of that step's stage completes once those MMAs have finished.
+    int h_stage0 = -1, h_stage1 = -1;
+    uint32_t h_phase0 = 0, h_phase1 = 0;
     const int lr_slots = (r + kLrChunk - 1) / kLrChunk;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
       for (int c = 0; c < lr_slots; ++c)
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       for (int kt = 0; kt < args.k_iters; ++kt) {
-        bool got = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
-        got = got && mbar_wait_bounded(sf_free_bar(sfb), sf_phase ^ 1u, wait_ns, status, kStatusEpilogue, abort_flag);
+        const bool got_data = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
+        if (!__all_sync(0xffffffffu, got_data)) { ok = false; break; }
+        // read the stage's scale atoms now; only the TMEM stores wait for the buffer
+        const uint8_t* sfs = smem + stage * L::kStage + L::kOffSfa + lane * 16;
+        uint4 fa[4], fb[4 * L::kSfAtomsB];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) fa[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
+#pragma unroll
+        for (int i = 0; i < 4 * L::kSfAtomsB; ++i)
+          fb[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + L::kOffSfb + lane * 16 + 512 * i);
+        bool got = true;
+        const int hs = sfb ? h_stage1 : h_stage0;
+        const uint32_t hp = sfb ? h_phase1 : h_phase0;
+        if (hs >= 0) got = mbar_wait_bounded(empty_bar(hs), hp, wait_ns, status, kStatusEpilogue, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
-        const uint8_t* sfs = smem + stage * L::kStage + L::kOffSfa + lane * 16;
         const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kColSf + sfb * L::kSfCols;
-        uint4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
-        tmem_st_x16(tsf, v);
+        tmem_st_x16(tsf, fa);
 #pragma unroll
         for (int h = 0; h < L::kSfAtomsB; ++h) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            v[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + L::kOffSfb + lane * 16 + 512 * (4 * h + i));
+          const uint4 v[4] = {fb[4 * h], fb[4 * h + 1], fb[4 * h + 2], fb[4 * h + 3]};
           tmem_st_x16(tsf + 16 + 16 * h, v);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(sf_full_bar(sfb));
+        if (sfb) {
+          h_stage1 = stage;
+          h_phase1 = phase;
+        } else {
+          h_stage0 = stage;
+          h_phase0 = phase;
+        }
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         if (++sfb == 2) { sfb = 0; sf_phase ^= 1u; }
       }
