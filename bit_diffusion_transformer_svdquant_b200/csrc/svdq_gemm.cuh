@@ -198,80 +198,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    // Measured on B200: the tensor pipe takes one tcgen05 instruction at a time (>= 64 cycles each,
-    // N/2 cycles for an NVFP4 MMA), and the next MMA issue returns only when the previous MMA is done,
-    // so the issuing thread's other work overlaps only the one MMA in flight. Per K step it therefore
-    // does one commit (which also frees the step's scale buffer: the writers watch the stage release)
-    // and waits for the next step's scales between the third and fourth MMA. A K step waits only on
-    // its scale buffer: the writers arrive there after they have seen the stage's data land.
-    if (lane == 0) {
-      const int num_tiles = args.num_tiles, k_iters = args.k_iters;
-      const int rc = r < kLrChunk ? r : kLrChunk;
-      const int nj = rc >> 4;
-      const uint32_t idesc_fp4 = idesc_nvfp4(128, N_TILE);
-      const uint32_t idesc_lr = idesc_bf16(128, N_TILE);
-      // descriptor halves: low = start address / 16 | LBO (16 B) / 16 << 16; high = SBO / 16 |
-      // version 1 | swizzle mode << 29
-      const uint32_t lo0 = (sbase >> 4) | (1u << 16);
-      const uint32_t hi_ab = (1024u >> 4) | (1u << 14) | (2u << 29);
-      const uint32_t hi_lr = ((8u * rc * 2u) >> 4) | (1u << 14) | (lr_swizzle_mode(rc) << 29);
-      const uint32_t tsf0 = tmem + L::kColSf;
-      int stage = 0, sfb = 0, acc = 0;
-      uint32_t phase = 0, sf_phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        if (!(ok = mbar_wait_bounded(acce_bar(acc), acc_phase ^ 1u, wait_ns, status, kStatusMma, abort_flag))) break;
-        const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
-        uint32_t accumulate = 0;
-        for (int c0 = 0; c0 < r; c0 += kLrChunk) {
-          if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t lo = lo0 + stage * (L::kStage >> 4);
-          for (int j = 0; j < nj; ++j) {
-            mma_bf16(d, desc_join(lo + 2u * j, hi_lr), desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr), idesc_lr,
-                     accumulate);
-            mma_bf16(d, desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr), desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr),
-                     idesc_lr, 1u);
-            accumulate = 1;
-          }
-          tc_commit(empty_bar(stage));
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        // the tile's first K step: its scales
-        if (!(ok = mbar_wait_bounded(sf_full_bar(sfb), sf_phase, wait_ns, status, kStatusMma, abort_flag))) break;
+    // Per K step: wait for the step's scale buffer (the writers arrive there only after they have
+    // seen the stage's data land), 4 MMAs, one commit that releases the stage (the writers also take
+    // it as the release of the scale buffer used two steps back).
+    // The whole warp runs this loop (warp-uniform operands); elect.sync inside the MMA and commit
+    // helpers picks the issuing lane, and a wait succeeds only when it succeeds in every lane.
+    auto wait_all = [&](uint32_t bar, uint32_t parity, unsigned code, volatile int* abort_ptr) {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, wait_ns, status, code, abort_ptr));
+    };
+    const int num_tiles = args.num_tiles, k_iters = args.k_iters;
+    const int rc = r < kLrChunk ? r : kLrChunk;
+    const int nj = rc >> 4;
+    const uint32_t idesc_fp4 = idesc_nvfp4(128, N_TILE);
+    const uint32_t idesc_lr = idesc_bf16(128, N_TILE);
+    // descriptor halves: low = start address / 16 | LBO (16 B) / 16 << 16; high = SBO / 16 |
+    // version 1 | swizzle mode << 29
+    const uint32_t lo0 = (sbase >> 4) | (1u << 16);
+    const uint32_t hi_ab = (1024u >> 4) | (1u << 14) | (2u << 29);
+    const uint32_t hi_lr = ((8u * rc * 2u) >> 4) | (1u << 14) | (lr_swizzle_mode(rc) << 29);
+    const uint32_t tsf0 = tmem + L::kColSf;
+    int stage = 0, sfb = 0, acc = 0;
+    uint32_t phase = 0, sf_phase = 0, acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      if (!(ok = wait_all(acce_bar(acc), acc_phase ^ 1u, kStatusMma, abort_flag))) break;
+      const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
+      uint32_t accumulate = 0;
+      for (int c0 = 0; c0 < r; c0 += kLrChunk) {
+        if (!(ok = wait_all(full_bar(stage), phase, kStatusMma, abort_flag))) break;
         tc_fence_after();
-        for (int kt = 0; kt < k_iters; ++kt) {
-          const uint32_t la = lo0 + stage * (L::kStage >> 4);
-          const uint32_t lb = la + (L::kOffB >> 4);
-          const uint32_t tsf = tsf0 + sfb * L::kSfCols;
-          mma_nvfp4(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_fp4, tsf, tsf + 16, accumulate);
-          mma_nvfp4(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_fp4, tsf + 4,
-                    tsf + 16 + 4 * L::kSfAtomsB, 1u);
-          mma_nvfp4(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_fp4, tsf + 8,
-                    tsf + 16 + 8 * L::kSfAtomsB, 1u);
+        const uint32_t lo = lo0 + stage * (L::kStage >> 4);
+        for (int j = 0; j < nj; ++j) {
+          const uint64_t bl = desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr);
+          mma_bf16_warp(d, desc_join(lo + 2u * j, hi_lr), bl, idesc_lr, accumulate);
+          mma_bf16_warp(d, desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr), bl, idesc_lr, 1u);
           accumulate = 1;
-          const int nsfb = sfb ^ 1;
-          const uint32_t nsf_phase = sf_phase ^ static_cast<uint32_t>(sfb);
-          if (kt + 1 < k_iters)
-            ok = mbar_wait_bounded(sf_full_bar(nsfb), nsf_phase, wait_ns, status, kStatusMma, abort_flag);
-          tc_fence_after();
-          mma_nvfp4(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_fp4, tsf + 12,
-                    tsf + 16 + 12 * L::kSfAtomsB, 1u);
-          tc_commit(empty_bar(stage));
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          sfb = nsfb;
-          sf_phase = nsf_phase;
-          if (!ok) break;
         }
-        if (!ok) break;
-        tc_commit(accf_bar(acc));
-        if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+        tc_commit_warp(empty_bar(stage));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      // Drain: all issued MMAs complete before TMEM is freed.
-      tc_commit(drain_bar);
-      mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
+      if (!ok) break;
+      for (int kt = 0; kt < k_iters; ++kt) {
+        // The wait sits before the step's first MMA: placed between queued MMAs, a barrier wait
+        // measurably stalled the tensor pipe on B200.
+        if (!(ok = wait_all(sf_full_bar(sfb), sf_phase, kStatusMma, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t la = lo0 + stage * (L::kStage >> 4);
+        const uint32_t lb = la + (L::kOffB >> 4);
+        const uint32_t tsf = tsf0 + sfb * L::kSfCols;
+        mma_nvfp4_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_fp4, tsf, tsf + 16, accumulate);
+        mma_nvfp4_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_fp4, tsf + 4,
+                       tsf + 16 + 4 * L::kSfAtomsB, 1u);
+        mma_nvfp4_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_fp4, tsf + 8,
+                       tsf + 16 + 8 * L::kSfAtomsB, 1u);
+        mma_nvfp4_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_fp4, tsf + 12,
+                       tsf + 16 + 12 * L::kSfAtomsB, 1u);
+        accumulate = 1;
+        tc_commit_warp(empty_bar(stage));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++sfb == 2) { sfb = 0; sf_phase ^= 1u; }
+      }
+      if (!ok) break;
+      tc_commit_warp(accf_bar(acc));
+      if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
+    // Drain: all issued MMAs complete before TMEM is freed.
+    tc_commit_warp(drain_bar);
+    wait_all(drain_bar, 0, kStatusDrain, nullptr);
   } else if (warp >= 6) {
     // ------------------------------------------------------------------ scale-factor writers (warps 6..9)
     // Each warp owns one TMEM lane quadrant and writes into it the replicated scale-factor layout
