@@ -46,14 +46,16 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct DeviceState {
   bool ready = false;
   int sm_count = 0;
+  int max_pairs[3] = {0, 0, 0};  // co-resident CTA pairs of the GEMM kernel for n_tile 256, 192, 128
   svdq_status status = SVDQ_OK;
   std::string error;
 };
 std::mutex g_dev_mu;
 DeviceState g_dev[64];
 
-constexpr int kStagesTile192 = 4;
-constexpr int kStagesTile128 = 5;
+constexpr int kStagesTile256 = 5;
+constexpr int kStagesTile192 = 5;
+constexpr int kStagesTile128 = 6;
 
 using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -82,6 +84,9 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
         return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
       g_encode = reinterpret_cast<Encode>(fn);
     }
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<256, kStagesTile256>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::GemmLayout<256, kStagesTile256>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<192, kStagesTile192>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<192, kStagesTile192>::kSmem));
@@ -96,6 +101,31 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
                                    svdq::QuantLayout<32>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::QuantLayout<64>::kSmem));
+    // How many CTA pairs of each GEMM instantiation can be resident at once: the persistent grid
+    // never asks for more (pairs must sit on two SMs of one GPC, so this can be below sms / 2).
+    auto max_pairs = [&](const void* fn, int smem, int* out) -> svdq_status {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+      cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
+      cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+      int n = 0;
+      SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, fn, &cfg));
+      if (n <= 0) return fail(SVDQ_ERR_CUDA, "GEMM kernel cannot be resident as CTA pairs");
+      *out = n;
+      return SVDQ_OK;
+    };
+    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::svdq_gemm_kernel<256, kStagesTile256>),
+                                  svdq::GemmLayout<256, kStagesTile256>::kSmem, &st.max_pairs[0]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::svdq_gemm_kernel<192, kStagesTile192>),
+                                  svdq::GemmLayout<192, kStagesTile192>::kSmem, &st.max_pairs[1]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::svdq_gemm_kernel<128, kStagesTile128>),
+                                  svdq::GemmLayout<128, kStagesTile128>::kSmem, &st.max_pairs[2]);
+        s != SVDQ_OK)
+      return s;
     st.sm_count = sms;
     st.ready = true;
   }
@@ -121,12 +151,15 @@ CUtensorMapSwizzle lr_swizzle(int r) { return r == 16 ? CU_TENSOR_MAP_SWIZZLE_32
 
 bool valid_r(int r) { return r == 0 || r == 16 || r == 32 || r == 64; }
 
+// GEMM tile width along N: 256 where it divides N (the widest MMA: fewest bytes streamed per
+// flop), else 192, else 128. SVDQ_N_TILE overrides it with another valid width.
 int choose_n_tile(int N) {
   const char* env = getenv("SVDQ_N_TILE");
   if (env != nullptr) {
     const int t = atoi(env);
-    if ((t == 128 || t == 192) && N % t == 0) return t;
+    if ((t == 256 || t == 192 || t == 128) && N % t == 0) return t;
   }
+  if (N % 256 == 0) return 256;
   if (N % 192 == 0) return 192;
   if (N % 128 == 0) return 128;
   return 0;
@@ -301,13 +334,14 @@ svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const ui
   static_assert(sizeof(w.tmap) >= 2 * sizeof(CUtensorMap), "tmap storage");
   CUtensorMap tmB, tmL2;
   std::memset(&tmL2, 0, sizeof(tmL2));
-  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K / 2, N, K / 2, 128, n_tile,
+  // each CTA of a GEMM pair stages half of a tile's n_tile rows
+  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K / 2, N, K / 2, 128, n_tile / 2,
                                 CU_TENSOR_MAP_SWIZZLE_128B);
       s != SVDQ_OK)
     return s;
   if (r > 0) {
     if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, N, static_cast<uint64_t>(r) * 2,
-                                  r < 32 ? r : 32, n_tile, lr_swizzle(r));
+                                  r < 32 ? r : 32, n_tile / 2, lr_swizzle(r));
         s != SVDQ_OK)
       return s;
   }
@@ -420,7 +454,8 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
   if (!swiglu && w->swiglu_interleaved) return fail(SVDQ_ERR_INVALID_ARG, "weight packed for SwiGLU");
   if (!aligned16(Y) || (bias != nullptr && !aligned16(bias))) return fail(SVDQ_ERR_UNSUPPORTED, "Y / bias alignment");
   const int n_tile = w->n_tile;
-  if ((n_tile != 192 && n_tile != 128) || w->N % n_tile != 0) return fail(SVDQ_ERR_UNSUPPORTED, "bad n_tile");
+  if ((n_tile != 256 && n_tile != 192 && n_tile != 128) || w->N % n_tile != 0)
+    return fail(SVDQ_ERR_UNSUPPORTED, "bad n_tile");
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
 
@@ -454,9 +489,10 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
   g.K = K;
   g.r = r;
   g.m_tiles = act->M_pad / 128;
+  g.m_pairs = (g.m_tiles + 1) / 2;
   g.n_tiles = w->N / n_tile;
   g.k_iters = K / 256;
-  g.num_tiles = g.m_tiles * g.n_tiles;
+  g.num_tiles = g.m_pairs * g.n_tiles;
   g.ldy = swiglu ? w->N / 2 : w->N;
   g.out_f32 = out_dtype == SVDQ_OUT_F32 ? 1 : 0;
   g.epi = static_cast<int>(epi);
@@ -467,9 +503,18 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
                                 g.out_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
       s != SVDQ_OK)
     return s;
-  const int grid = g.num_tiles < sms ? g.num_tiles : sms;
+  int max_pairs = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    max_pairs = g_dev[dev].max_pairs[n_tile == 256 ? 0 : n_tile == 192 ? 1 : 2];
+  }
+  const int pairs = g.num_tiles < max_pairs ? g.num_tiles : max_pairs;
+  const dim3 grid(2 * pairs);  // clusters of 2 CTAs (compiled into the kernel)
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (n_tile == 192) {
+  if (n_tile == 256) {
+    svdq::svdq_gemm_kernel<256, kStagesTile256><<<grid, svdq::kGemmThreads, svdq::GemmLayout<256, kStagesTile256>::kSmem, st>>>(
+        tmA, tmB, tmU, tmL2, tmY, g);
+  } else if (n_tile == 192) {
     svdq::svdq_gemm_kernel<192, kStagesTile192><<<grid, svdq::kGemmThreads, svdq::GemmLayout<192, kStagesTile192>::kSmem, st>>>(
         tmA, tmB, tmU, tmL2, tmY, g);
   } else {

@@ -7,26 +7,39 @@
 // scale applies at the end. The fused QKV / SwiGLU epilogues follow the fused NVFP4 GEMMs of
 // "FLUX 3 Image Klein on NVIDIA Blackwell", method 1.
 //
-// Structure (one persistent CTA per SM, 6 warps):
-//   warp 0      TMA producer: per 256-wide K step, A (128 x 128 B) and B (n_tile x 128 B) codes as
-//               128B-swizzled 2-D tiles, plus the matching scale-factor atoms as 1-D bulk copies,
-//               into a STAGES-deep shared-memory ring (full/empty mbarriers). Before a tile's K
-//               loop, ring slots carry the tile's U_hi, U_lo (128 x r) and L2^T (n_tile x r) in
-//               chunks of 32 columns of r.
-//   warp 1      TMEM allocator + single-thread MMA issuer:
-//               4 x tcgen05.mma kind::mxf4nvf4 (M=128, N=n_tile, K=64) per K step, 2 r/16 x
-//               kind::f16 (hi and lo halves of U against the same L2 tile) for the low-rank term; tcgen05.commit frees ring slots and publishes
-//               finished accumulators. Accumulators are double-buffered in TMEM when they fit.
-//   warps 2..5  epilogue: tcgen05.ld (each warp its 32-lane quadrant), y = alpha acc (+ bias),
-//               SwiGLU on interleaved gate/up columns, bf16 or fp32 store.
-//   warps 6..9  scale-factor writers: per K step, copy the stage's E4M3 scale atoms from shared
-//               memory into a double-buffered TMEM region with tcgen05.st (each warp its lane
-//               quadrant). Measured on B200, every tcgen05.cp costs ~64 tensor-pipe cycles whatever
-//               its shape, so copying 12 atoms per K step with tcgen05.cp starved the MMAs; stores
-//               from four warps run beside the MMAs without slowing them.
+// Structure: persistent clusters of two CTAs (one per SM) that share each 256 x n_tile output tile
+// through the CTA-pair form of the tensor-core MMA (cta_group::2): the even CTA issues every MMA of
+// the pair; rows 0..127 of A, of the accumulator and of the output belong to the even CTA, rows
+// 128..255 to the odd one, and each CTA stages half of B's n_tile rows. Per CTA (14 warps):
+//   warp 0       TMA producer: per 256-wide K step, its 128 A rows and n_tile/2 B rows (128B-
+//                swizzled 2-D tiles) plus the scale-factor atoms (its own 128 A rows; all n_tile B
+//                rows) as 1-D bulk copies, into a STAGES-deep ring on this CTA's own barriers.
+//                Before a tile's K loop, ring slots carry U_hi, U_lo (its 128 rows) and its half
+//                of L2^T in chunks of 32 columns of r.
+//   warp 1       TMEM allocation for the pair; in the even CTA also the MMA issuer: per ring slot
+//                it waits for the slot's barrier in the even CTA (8 arrivals: the scale writers of
+//                both CTAs), issues 4 x tcgen05.mma kind::mxf4nvf4 (M=256, N=n_tile, K=64) or the
+//                low-rank kind::f16 MMAs, and multicasts one commit to the slot's empty barrier in
+//                both CTAs.
+//   warps 2..9   epilogue: two warps per 32-lane TMEM quadrant, each half of the tile's columns:
+//                tcgen05.ld, y = alpha acc (+ bias), SwiGLU on interleaved gate/up columns, into a
+//                swizzled staging buffer, TMA store. The accumulator goes back to the issuer (a
+//                remote arrive) as soon as its last columns are in registers.
+//   warps 10..13 scale-factor writers: per ring slot, wait for this CTA's data, copy the scale
+//                atoms from shared memory into one of 4 TMEM scale buffers with tcgen05.st (each
+//                warp its lane quadrant), then arrive on the issuer's barrier in the even CTA.
+//                Measured on B200, every tcgen05.cp costs ~64 tensor-pipe cycles whatever its
+//                shape, so copying 12 atoms per K step with tcgen05.cp starved the MMAs; stores
+//                from four warps run beside the MMAs without slowing them.
+// TMEM (512 columns): the accumulator (n_tile columns; two buffers when n_tile = 128) and 4 scale
+// buffers of 16 + 16 * ceil(n_tile / 128) columns. Measured on B200: with only 2 scale buffers
+// the commit -> writer -> remote arrive -> issuer round trip (~900 cycles across the pair) could
+// not hide under one K step; and one CTA per 128 x 192 tile had to stream 48 KB per 384-cycle K
+// step from L2 per SM, above what a B200 SM sustained in isolation (~75-90 B per cycle), against
+// 38 KB per 512 cycles here.
 // Every mbarrier wait is bounded (global timer); a wait that runs out records a status bit, sets
-// a shared abort flag so that the other roles stop too, and the kernel drains its own copies and
-// MMAs before freeing TMEM and returning.
+// a shared abort flag so that the other roles of the CTA stop too, and the kernel drains its own
+// copies and MMAs before the cluster-wide barrier that precedes freeing TMEM.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -45,14 +58,15 @@ struct GemmArgs {
   void* Y;
   unsigned long long wait_ns;
   int M, M_pad, N, K, r;
-  int m_tiles, n_tiles, k_iters, num_tiles;
-  int ldy, out_f32, epi;  // epi bit 0: bias, bit 1: SwiGLU
+  int m_tiles, m_pairs, n_tiles, k_iters, num_tiles;  // num_tiles = m_pairs * n_tiles pair tiles
+  int ldy, out_f32, epi;                              // epi bit 0: bias, bit 1: SwiGLU
 };
 
 template <int N_TILE, int STAGES>
 struct GemmLayout {
+  static constexpr int kBRows = N_TILE / 2;  // rows of B staged by each CTA of the pair
   static constexpr int kA = 128 * 128;
-  static constexpr int kB = N_TILE * 128;
+  static constexpr int kB = kBRows * 128;
   static constexpr int kSfAtomsB = (N_TILE + 127) / 128;
   static constexpr int kSfa = 4 * 512;
   static constexpr int kSfb = 4 * kSfAtomsB * 512;
@@ -62,21 +76,25 @@ struct GemmLayout {
   static constexpr int kOffSfb = kA + kB + kSfa;
   // TMEM scale-factor buffer (one K step): SFA 4 MMAs x 4 columns, then SFB 4 MMAs x 4 x atoms.
   static constexpr int kSfCols = 16 + 16 * kSfAtomsB;
-  static constexpr int kAccBufs = (2 * N_TILE + 2 * kSfCols <= 512) ? 2 : 1;
-  static constexpr int kColSf = kAccBufs * N_TILE;  // two buffers of kSfCols columns from here
-  // epilogue staging: 4 warps x 2 buffers x (32 rows x 32 columns of fp32 at most)
-  static constexpr int kStageOut = 32 * 32 * 4;
+  static constexpr int kSfBufs = 4;
+  static constexpr int kAccBufs = (2 * N_TILE + kSfBufs * kSfCols <= 512) ? 2 : 1;
+  static constexpr int kColSf = kAccBufs * N_TILE;  // kSfBufs buffers of kSfCols columns from here
+  // epilogue staging: 8 warps x 4 KB (two 32 x 32 bf16 boxes or one fp32 box in flight)
+  static constexpr int kStageOutWarp = 4096;
   static constexpr int kOutOff = STAGES * kStage;
-  static constexpr int kBarOff = kOutOff + 4 * 2 * kStageOut;
-  static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1 + 4;
+  static constexpr int kBarOff = kOutOff + 8 * kStageOutWarp;
+  // full[STAGES], empty[STAGES], accf[kAccBufs], acce[kAccBufs], drain, sf_full[kSfBufs]
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1 + kSfBufs;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
-  static_assert(kColSf + 2 * kSfCols <= 512, "TMEM budget");
+  static_assert(kColSf + kSfBufs * kSfCols <= 512, "TMEM budget");
+  static_assert(kSfBufs <= STAGES, "a scale buffer's previous slot must still own its ring stage");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-// Low-rank operands move in chunks of rc = min(r, 32) columns: U_hi, U_lo (128 x rc each) and
-// L2^T (n_tile x rc), all bf16 with rc*2-byte rows (32B or 64B swizzle), one ring slot per chunk.
+// Low-rank operands move in chunks of rc = min(r, 32) columns: U_hi, U_lo (128 x rc each) and this
+// CTA's half of L2^T (n_tile/2 x rc), all bf16 with rc*2-byte rows (32B or 64B swizzle), one ring
+// slot per chunk.
 constexpr int kLrChunk = 32;
 constexpr int kOffULo = 128 * kLrChunk * 2;
 __device__ __forceinline__ uint32_t lr_swizzle_mode(int rc) { return rc == 16 ? 6u : 4u; }
@@ -89,46 +107,56 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint4 (&v)[4])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t num_clusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
 
-constexpr int kGemmThreads = 320;
+constexpr int kGemmThreads = 448;
 
 template <int N_TILE, int STAGES>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     svdq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
                      const __grid_constant__ CUtensorMap tmY, const GemmArgs args) {
   using L = GemmLayout<N_TILE, STAGES>;
+  constexpr int kSfBufs = L::kSfBufs, kAccBufs = L::kAccBufs;
   extern __shared__ uint8_t smem_raw[];
+  // the same offsets in both CTAs: the pair MMA addresses the odd CTA's operands by this CTA's
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + L::kBarOff;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
-  auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kAccBufs + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * L::kAccBufs);
-  auto sf_full_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * L::kAccBufs + 1 + b); };
-  auto sf_free_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * L::kAccBufs + 3 + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + kAccBufs + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * kAccBufs);
+  auto sf_full_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * kAccBufs + 1 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = args.r;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the pair's MMAs
+  const int pair0 = static_cast<int>(cluster_id_x()), npairs = static_cast<int>(num_clusters_x());
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < L::kAccBufs; ++b) {
+    for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 4);
+      mbar_init(acce_bar(b), 16);  // 8 epilogue warps in each CTA
     }
     mbar_init(drain_bar, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(sf_full_bar(b), 4);
-      mbar_init(sf_free_bar(b), 1);
-    }
+    for (int b = 0; b < kSfBufs; ++b) mbar_init(sf_full_bar(b), 8);  // 4 writer warps in each CTA
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmA);
@@ -140,11 +168,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), 512);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_addr(tmem_slot), 512);
+    tmem_relinquish_pair();
   }
+  // both CTAs' barriers are initialised before any remote arrive
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   unsigned* status = &g_svdq_status;
@@ -156,11 +185,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       const int rc = r < kLrChunk ? r : kLrChunk;
-      const uint32_t lr_bytes = static_cast<uint32_t>((2 * 128 + N_TILE) * rc * 2);
+      const uint32_t lr_bytes = static_cast<uint32_t>((2 * 128 + L::kBRows) * rc * 2);
       const int sf_row_stride = args.K >> 6;  // 64-wide K atoms per 128-row block
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-        const int m_blk = tile % args.m_tiles, n_blk = tile / args.m_tiles;
+      for (int tile = pair0; ok && tile < args.num_tiles; tile += npairs) {
+        const int m_pair = tile % args.m_pairs, n_blk = tile / args.m_pairs;
+        const int m_blk = 2 * m_pair + static_cast<int>(rank);
+        // an odd CTA past the last 128-row block loads zero-filled codes (rows past the tensor) and
+        // the last block's scales; none of its rows are stored
+        const int m_sf = m_blk < args.m_tiles ? m_blk : args.m_tiles - 1;
+        const int b_row = n_blk * N_TILE + static_cast<int>(rank) * L::kBRows;
         for (int c0 = 0; c0 < r; c0 += kLrChunk) {
           if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
             break;
@@ -168,13 +202,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(full_bar(stage), lr_bytes);
           tma_load_2d(sa, &tmU, c0, m_blk * 128, full_bar(stage));
           tma_load_2d(sa + kOffULo, &tmU, c0, args.M_pad + m_blk * 128, full_bar(stage));
-          tma_load_2d(sa + L::kOffB, &tmL2, c0, n_blk * N_TILE, full_bar(stage));
+          tma_load_2d(sa + L::kOffB, &tmL2, c0, b_row, full_bar(stage));
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        const uint8_t* sfa_tile = args.sfa + (static_cast<size_t>(m_blk) * sf_row_stride << 9);
+        const uint8_t* sfa_tile = args.sfa + (static_cast<size_t>(m_sf) * sf_row_stride << 9);
         const uint8_t* sfb_tile = args.sfb + (static_cast<size_t>(n_blk) * sf_row_stride * L::kSfAtomsB << 9);
         for (int kt = 0; kt < args.k_iters; ++kt) {
           if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
@@ -182,7 +216,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sa = sbase + stage * L::kStage;
           mbar_arrive_expect_tx(full_bar(stage), L::kStage);
           tma_load_2d(sa, &tmA, kt * 128, m_blk * 128, full_bar(stage));
-          tma_load_2d(sa + L::kOffB, &tmB, kt * 128, n_blk * N_TILE, full_bar(stage));
+          tma_load_2d(sa + L::kOffB, &tmB, kt * 128, b_row, full_bar(stage));
           bulk_load(sa + L::kOffSfa, sfa_tile + (static_cast<size_t>(kt) * 4 << 9), L::kSfa, full_bar(stage));
           bulk_load(sa + L::kOffSfb, sfb_tile + (static_cast<size_t>(kt) * 4 * L::kSfAtomsB << 9), L::kSfb,
                     full_bar(stage));
@@ -197,264 +231,333 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Per K step: wait for the step's scale buffer (the writers arrive there only after they have
-    // seen the stage's data land), 4 MMAs, one commit that releases the stage (the writers also take
-    // it as the release of the scale buffer used two steps back).
-    // The whole warp runs this loop (warp-uniform operands); elect.sync inside the MMA and commit
-    // helpers picks the issuing lane, and a wait succeeds only when it succeeds in every lane.
-    auto wait_all = [&](uint32_t bar, uint32_t parity, unsigned code, volatile int* abort_ptr) {
-      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, wait_ns, status, code, abort_ptr));
-    };
-    const int num_tiles = args.num_tiles, k_iters = args.k_iters;
-    const int rc = r < kLrChunk ? r : kLrChunk;
-    const int nj = rc >> 4;
-    const uint32_t idesc_fp4 = idesc_nvfp4(128, N_TILE);
-    const uint32_t idesc_lr = idesc_bf16(128, N_TILE);
-    // descriptor halves: low = start address / 16 | LBO (16 B) / 16 << 16; high = SBO / 16 |
-    // version 1 | swizzle mode << 29
-    const uint32_t lo0 = (sbase >> 4) | (1u << 16);
-    const uint32_t hi_ab = (1024u >> 4) | (1u << 14) | (2u << 29);
-    const uint32_t hi_lr = ((8u * rc * 2u) >> 4) | (1u << 14) | (lr_swizzle_mode(rc) << 29);
-    const uint32_t tsf0 = tmem + L::kColSf;
-    int stage = 0, sfb = 0, acc = 0;
-    uint32_t phase = 0, sf_phase = 0, acc_phase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      if (!(ok = wait_all(acce_bar(acc), acc_phase ^ 1u, kStatusMma, abort_flag))) break;
-      const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
-      uint32_t accumulate = 0;
-      for (int c0 = 0; c0 < r; c0 += kLrChunk) {
-        if (!(ok = wait_all(full_bar(stage), phase, kStatusMma, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t lo = lo0 + stage * (L::kStage >> 4);
-        for (int j = 0; j < nj; ++j) {
-          const uint64_t bl = desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr);
-          mma_bf16_warp(d, desc_join(lo + 2u * j, hi_lr), bl, idesc_lr, accumulate);
-          mma_bf16_warp(d, desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr), bl, idesc_lr, 1u);
-          accumulate = 1;
+    // ------------------------------------------------------------------ MMA issuer (even CTA)
+    // Per ring slot: wait for the slot's scale-buffer barrier (the writers of both CTAs arrive
+    // there only after they have seen their CTA's data land and have stored the step's scales),
+    // the MMAs, and one commit multicast to the slot's empty barrier in both CTAs (the writers also
+    // take it as the release of the scale buffer that slot used). The wait sits before the slot's
+    // first MMA: placed between queued MMAs, a barrier wait measurably stalled the tensor pipe on
+    // B200. The whole warp runs this loop (warp-uniform operands); elect.sync inside the MMA and
+    // commit helpers picks the issuing lane, and a wait succeeds only when it succeeds in every lane.
+    if (rank == 0) {
+      auto wait_all = [&](uint32_t bar, uint32_t parity, unsigned code, volatile int* abort_ptr) {
+        return __all_sync(0xffffffffu, mbar_wait_bounded_cluster(bar, parity, wait_ns, status, code, abort_ptr));
+      };
+      const int num_tiles = args.num_tiles, k_iters = args.k_iters;
+      const int rc = r < kLrChunk ? r : kLrChunk;
+      const int nj = rc >> 4;
+      const uint32_t idesc_fp4 = idesc_nvfp4(256, N_TILE);
+      const uint32_t idesc_lr = idesc_bf16(256, N_TILE);
+      // descriptor halves: low = start address / 16 | LBO (16 B) / 16 << 16; high = SBO / 16 |
+      // version 1 | swizzle mode << 29
+      const uint32_t lo0 = (sbase >> 4) | (1u << 16);
+      const uint32_t hi_ab = (1024u >> 4) | (1u << 14) | (2u << 29);
+      const uint32_t hi_lr = ((8u * rc * 2u) >> 4) | (1u << 14) | (lr_swizzle_mode(rc) << 29);
+      const uint32_t tsf0 = tmem + L::kColSf;
+      constexpr uint16_t kBoth = 3;
+      int stage = 0, sfb = 0, acc = 0;
+      uint32_t phase = 0, sf_phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair0; ok && tile < num_tiles; tile += npairs) {
+        if (!(ok = wait_all(acce_bar(acc), acc_phase ^ 1u, kStatusMma, abort_flag))) break;
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
+        uint32_t accumulate = 0;
+        for (int c0 = 0; c0 < r; c0 += kLrChunk) {
+          if (!(ok = wait_all(sf_full_bar(sfb), sf_phase, kStatusMma, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t lo = lo0 + stage * (L::kStage >> 4);
+          for (int j = 0; j < nj; ++j) {
+            const uint64_t bl = desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr);
+            mma_bf16_pair_warp(d, desc_join(lo + 2u * j, hi_lr), bl, idesc_lr, accumulate);
+            mma_bf16_pair_warp(d, desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr), bl, idesc_lr, 1u);
+            accumulate = 1;
+          }
+          tc_commit_pair_mc_warp(empty_bar(stage), kBoth);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++sfb == kSfBufs) { sfb = 0; sf_phase ^= 1u; }
         }
-        tc_commit_warp(empty_bar(stage));
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (!ok) break;
+        for (int kt = 0; kt < k_iters; ++kt) {
+          if (!(ok = wait_all(sf_full_bar(sfb), sf_phase, kStatusMma, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t la = lo0 + stage * (L::kStage >> 4);
+          const uint32_t lb = la + (L::kOffB >> 4);
+          const uint32_t tsf = tsf0 + sfb * L::kSfCols;
+          mma_nvfp4_pair_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_fp4, tsf, tsf + 16, accumulate);
+          mma_nvfp4_pair_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_fp4, tsf + 4,
+                              tsf + 16 + 4 * L::kSfAtomsB, 1u);
+          mma_nvfp4_pair_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_fp4, tsf + 8,
+                              tsf + 16 + 8 * L::kSfAtomsB, 1u);
+          mma_nvfp4_pair_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_fp4, tsf + 12,
+                              tsf + 16 + 12 * L::kSfAtomsB, 1u);
+          accumulate = 1;
+          tc_commit_pair_mc_warp(empty_bar(stage), kBoth);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++sfb == kSfBufs) { sfb = 0; sf_phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc_warp(accf_bar(acc), kBoth);
+        if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
-      if (!ok) break;
-      for (int kt = 0; kt < k_iters; ++kt) {
-        // The wait sits before the step's first MMA: placed between queued MMAs, a barrier wait
-        // measurably stalled the tensor pipe on B200.
-        if (!(ok = wait_all(sf_full_bar(sfb), sf_phase, kStatusMma, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t la = lo0 + stage * (L::kStage >> 4);
-        const uint32_t lb = la + (L::kOffB >> 4);
-        const uint32_t tsf = tsf0 + sfb * L::kSfCols;
-        mma_nvfp4_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_fp4, tsf, tsf + 16, accumulate);
-        mma_nvfp4_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_fp4, tsf + 4,
-                       tsf + 16 + 4 * L::kSfAtomsB, 1u);
-        mma_nvfp4_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_fp4, tsf + 8,
-                       tsf + 16 + 8 * L::kSfAtomsB, 1u);
-        mma_nvfp4_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_fp4, tsf + 12,
-                       tsf + 16 + 12 * L::kSfAtomsB, 1u);
-        accumulate = 1;
-        tc_commit_warp(empty_bar(stage));
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        if (++sfb == 2) { sfb = 0; sf_phase ^= 1u; }
-      }
-      if (!ok) break;
-      tc_commit_warp(accf_bar(acc));
-      if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+      // Drain: all issued MMAs complete before TMEM may be freed.
+      tc_commit_pair_mc_warp(drain_bar, 1);
+      __all_sync(0xffffffffu, mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr));
     }
-    // Drain: all issued MMAs complete before TMEM is freed.
-    tc_commit_warp(drain_bar);
-    wait_all(drain_bar, 0, kStatusDrain, nullptr);
-  } else if (warp >= 6) {
-    // ------------------------------------------------------------------ scale-factor writers (warps 6..9)
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------------ scale-factor writers (warps 10..13)
     // Each warp owns one TMEM lane quadrant and writes into it the replicated scale-factor layout
     // the block-scaled MMA reads: for a 128-row atom, lane l, column c holds the 4 E4M3 scales of
-    // row l + 32 c -- exactly bytes [16 l, 16 l + 16) of the 512-byte atom in shared memory.
+    // row l + 32 c -- exactly bytes [16 l, 16 l + 16) of the 512-byte atom in shared memory. Every
+    // ring slot (low-rank chunks too, which carry no scales) is reported to the issuer's barrier.
     const int q = warp & 3;
-    int stage = 0, sfb = 0;
-    uint32_t phase = 0, sf_phase = 0;
-    // (stage, phase) of the last two K steps: buffer sfb was last read by the K step two back, and
-    // the MMA thread's release of that step's stage completes once those MMAs have finished.
-    int h_stage0 = -1, h_stage1 = -1;
-    uint32_t h_phase0 = 0, h_phase1 = 0;
+    int stage = 0, sfb = 0, slots_done = 0;
+    uint32_t phase = 0;
     const int lr_slots = (r + kLrChunk - 1) / kLrChunk;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-      for (int c = 0; c < lr_slots; ++c)
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-      for (int kt = 0; kt < args.k_iters; ++kt) {
+    for (int tile = pair0; ok && tile < args.num_tiles; tile += npairs) {
+      for (int slot = 0; slot < lr_slots + args.k_iters; ++slot) {
         const bool got_data = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
         if (!__all_sync(0xffffffffu, got_data)) { ok = false; break; }
+        const bool has_sf = slot >= lr_slots;
         // read the stage's scale atoms now; only the TMEM stores wait for the buffer
-        const uint8_t* sfs = smem + stage * L::kStage + L::kOffSfa + lane * 16;
         uint4 fa[4], fb[4 * L::kSfAtomsB];
+        if (has_sf) {
+          const uint8_t* sfs = smem + stage * L::kStage + L::kOffSfa + lane * 16;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) fa[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
+          for (int i = 0; i < 4; ++i) fa[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
 #pragma unroll
-        for (int i = 0; i < 4 * L::kSfAtomsB; ++i)
-          fb[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + L::kOffSfb + lane * 16 + 512 * i);
-        bool got = true;
-        const int hs = sfb ? h_stage1 : h_stage0;
-        const uint32_t hp = sfb ? h_phase1 : h_phase0;
-        if (hs >= 0) got = mbar_wait_bounded(empty_bar(hs), hp, wait_ns, status, kStatusEpilogue, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kColSf + sfb * L::kSfCols;
-        tmem_st_x16(tsf, fa);
-#pragma unroll
-        for (int h = 0; h < L::kSfAtomsB; ++h) {
-          const uint4 v[4] = {fb[4 * h], fb[4 * h + 1], fb[4 * h + 2], fb[4 * h + 3]};
-          tmem_st_x16(tsf + 16 + 16 * h, v);
+          for (int i = 0; i < 4 * L::kSfAtomsB; ++i)
+            fb[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + L::kOffSfb + lane * 16 + 512 * i);
         }
-        tmem_wait_st();
+        // Every slot, with scales or not, first waits for the release of the slot kSfBufs back (the
+        // previous one on barrier sfb, whose MMAs read this scale buffer): then no CTA can arrive
+        // for this slot while that slot's phase still waits for the other CTA's writers. That slot
+        // is at most STAGES back, so its ring stage has not been released a second time.
+        bool got = true;
+        if (slots_done >= kSfBufs) {
+          int ps = stage - kSfBufs;
+          uint32_t pp = phase;
+          if (ps < 0) {
+            ps += STAGES;
+            pp ^= 1u;
+          }
+          got = mbar_wait_bounded(empty_bar(ps), pp, wait_ns, status, kStatusEpilogue, abort_flag);
+        }
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        if (has_sf) {
+          tc_fence_after();
+          const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kColSf + sfb * L::kSfCols;
+          tmem_st_x16(tsf, fa);
+#pragma unroll
+          for (int h = 0; h < L::kSfAtomsB; ++h) {
+            const uint4 v[4] = {fb[4 * h], fb[4 * h + 1], fb[4 * h + 2], fb[4 * h + 3]};
+            tmem_st_x16(tsf + 16 + 16 * h, v);
+          }
+          tmem_wait_st();
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(sf_full_bar(sfb));
-        if (sfb) {
-          h_stage1 = stage;
-          h_phase1 = phase;
-        } else {
-          h_stage0 = stage;
-          h_phase0 = phase;
-        }
+        if (lane == 0) mbar_arrive_cluster(cluster_map(sf_full_bar(sfb), 0));
+        ++slots_done;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        if (++sfb == 2) { sfb = 0; sf_phase ^= 1u; }
+        if (++sfb == kSfBufs) sfb = 0;
       }
     }
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 2..5)
-    // Each warp drains its 32-lane TMEM quadrant 32 columns at a time, applies alpha / bias /
-    // SwiGLU, writes the 32 x 32 block into a swizzled shared-memory buffer (64B swizzle for bf16,
-    // 128B for fp32 rows: conflict-free 16-byte writes) and one lane stores it with a TMA tensor
-    // store; two buffers per warp let the next block fill while the previous store drains. Rows at
-    // or beyond M are clipped by the tensor map.
-    const int q = warp & 3;
+    // ------------------------------------------------------------------ epilogue (warps 2..9)
+    // Warp (q, h): TMEM lane quadrant q = warp % 4, half h of the tile's 32-column output chunks.
+    // A round loads up to 64 accumulator columns (tcgen05.ld), converts them (alpha, bias, SwiGLU;
+    // bf16 results stay packed in registers) and, after the last round's loads, hands the
+    // accumulator back before any store: the issuer's next tile then waits only for the loads.
+    // Each 32 x 32 output block goes through a swizzled staging box (64B swizzle for bf16 rows,
+    // 128B for fp32: conflict-free 16-byte writes) and a TMA tensor store that clips rows >= M.
+    const int q = warp & 3, h = (warp - 2) >> 2;
     const float alpha = *args.alpha;
     const bool has_bias = (args.epi & 1) != 0;
     const bool swiglu = (args.epi & 2) != 0;
     const bool f32 = args.out_f32 != 0;
     const int hN = args.N >> 1;
-    uint8_t* stage_out = smem + L::kOutOff + q * 2 * L::kStageOut;
-    int buf = 0;
+    uint8_t* stage_out = smem + L::kOutOff + (warp - 2) * L::kStageOutWarp;
+    // 32-column output chunks of a tile, split between the two warps of a quadrant
+    constexpr int kPlainPerWarp = N_TILE / 64;  // chunks per warp without SwiGLU
+    constexpr int kGluChunks = N_TILE / 64;     // output chunks per tile with SwiGLU
+    const int glu_beg = h * ((kGluChunks + 1) >> 1);
+    const int glu_end = h ? kGluChunks : ((kGluChunks + 1) >> 1);
     int acc = 0;
     uint32_t acc_phase = 0;
-    auto emit = [&](const float (&v)[32], int row0, int col0) {
-      // buffer reuse: the store issued from it two blocks ago has finished reading
-      if (lane == 0) bulk_wait_group_read<1>();
-      __syncwarp();
-      uint8_t* dst = stage_out + buf * L::kStageOut;
-      if (f32) {
-        // 128-byte rows, 8 chunks of 16 bytes; chunk j of row `lane` lives at j ^ (lane % 8)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4*>(dst + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-              make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      } else {
-        // 64-byte rows, 4 chunks; chunk j of row `lane` lives at j ^ ((lane / 2) % 4)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-            w[e] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          *reinterpret_cast<uint4*>(dst + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
+    // a staging box is reused once the store issued from it has finished reading
+    auto store_box = [&](uint8_t* dst, int row0, int col0) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         tma_store_2d(&tmY, smem_addr(dst), col0, row0);
         bulk_commit_group();
       }
-      buf ^= 1;
     };
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
-      const int m_blk = tile % args.m_tiles, n_blk = tile / args.m_tiles;
+    auto pack_bf16 = [&](const float (&v)[32], uint32_t (&pk)[16]) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+    };
+    // staging: two 2 KB bf16 boxes or one 4 KB fp32 box per warp; a box is rewritten once the
+    // store issued from it has finished reading it
+    auto write_box_bf16 = [&](const uint32_t (&pk)[16], int b) {
+      uint8_t* dst = stage_out + b * 2048;
+      // 64-byte rows, 4 chunks; chunk j of row `lane` lives at j ^ ((lane / 2) % 4)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(dst + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    };
+    auto boxes_free = [&]() {
+      if (lane == 0) bulk_wait_group_read<0>();
+      __syncwarp();
+    };
+    auto emit_f32 = [&](const float (&v)[32], int row0, int col0) {
+      uint8_t* dst = stage_out;
+      if (lane == 0) bulk_wait_group_read<0>();
+      __syncwarp();
+      // 128-byte rows, 8 chunks of 16 bytes; chunk j of row `lane` lives at j ^ (lane % 8)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(dst + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      store_box(dst, row0, col0);
+    };
+    // y = alpha * acc (+ bias) for 32 columns starting at output column n0 of the bias
+    auto affine = [&](float (&v)[32], int n0) {
+      if (has_bias) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          float b[8];
+          bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n0 + i)), b);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[i + j] = fmaf(alpha, v[i + j], b[j]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = alpha * v[i];
+      }
+    };
+    auto release_acc = [&]() {
+      // all of this warp's accumulator columns are in registers: hand the buffer back to the issuer
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_map(acce_bar(acc), 0));
+    };
+    for (int tile = pair0; tile < args.num_tiles; tile += npairs) {
+      const int m_pair = tile % args.m_pairs, n_blk = tile / args.m_pairs;
+      const int m_blk = 2 * m_pair + static_cast<int>(rank);
       // warp-uniform outcome: tcgen05.ld below is a .sync.aligned warp instruction
       const bool got = mbar_wait_bounded(accf_bar(acc), acc_phase, wait_ns, status, kStatusEpilogue, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int row0 = m_blk * 128 + q * 32;
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * N_TILE);
-      if (!swiglu) {
-#pragma unroll 1
-        for (int c = 0; c < N_TILE / 32; ++c) {
-          float v[32];
-          tmem_ld_32x32(tb + c * 32, v);
+      if (!swiglu && !f32) {
+        // bf16 out, 64 columns per load round: chunks 0 and 1 are scaled, packed and written into
+        // the two staging boxes, later chunks stay packed in registers; the accumulator is released
+        // after the last round's loads and only then are the boxes stored (measured on B200:
+        // staging and storing each chunk before the next load took ~700 cycles per chunk, all of it
+        // on the issuer's path to the next tile)
+        const int c_beg = h * kPlainPerWarp;
+        uint32_t pk[2][16];
+        boxes_free();
+#pragma unroll
+        for (int i = 0; i < kPlainPerWarp; i += 2) {
+          float v[2][32];
+          tmem_ld_32x32(tb + (c_beg + i) * 32, v[0]);
+          if (i + 1 < kPlainPerWarp) tmem_ld_32x32(tb + (c_beg + i + 1) * 32, v[1]);
           tmem_wait_ld();
-          if (c == N_TILE / 32 - 1) {
-            // all of this accumulator is in registers or already consumed: hand it back early
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acce_bar(acc));
-          }
-          const int n0 = n_blk * N_TILE + c * 32;
-          if (has_bias) {
+          if (i + 2 >= kPlainPerWarp) release_acc();
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              float b[8];
-              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n0 + i)), b);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) v[i + j] = fmaf(alpha, v[i + j], b[j]);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = alpha * v[i];
-          }
-          emit(v, row0, n0);
-        }
-      } else {
-        constexpr int kHalf = N_TILE / 2;
-#pragma unroll 1
-        for (int c = 0; c < kHalf / 32; ++c) {
-          float gt[32], up[32];
-          tmem_ld_32x32(tb + c * 32, gt);
-          tmem_ld_32x32(tb + kHalf + c * 32, up);
-          tmem_wait_ld();
-          if (c == kHalf / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acce_bar(acc));
-          }
-          const int j0 = n_blk * kHalf + c * 32;
-          if (has_bias) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              float bg[8], bu[8];
-              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + j0 + i)), bg);
-              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + hN + j0 + i)), bu);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                gt[i + j] = fmaf(alpha, gt[i + j], bg[j]);
-                up[i + j] = fmaf(alpha, up[i + j], bu[j]);
+          for (int u = 0; u < 2; ++u) {
+            const int j = i + u;
+            if (j < kPlainPerWarp) {
+              affine(v[u], n_blk * N_TILE + (c_beg + j) * 32);
+              if (j < 2) {
+                uint32_t t[16];
+                pack_bf16(v[u], t);
+                write_box_bf16(t, j);
+              } else {
+                pack_bf16(v[u], pk[j - 2]);
               }
             }
-          } else {
+          }
+        }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              gt[i] = alpha * gt[i];
-              up[i] = alpha * up[i];
+        for (int j = 0; j < kPlainPerWarp; ++j) {
+          if (j >= 2) {
+            // box j % 2 is free once the store issued from it two chunks ago has read it
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            write_box_bf16(pk[j - 2], j & 1);
+          }
+          store_box(stage_out + (j & 1) * 2048, row0, n_blk * N_TILE + (c_beg + j) * 32);
+        }
+      } else if (!swiglu) {
+        // fp32 out: chunk by chunk (the whole tile would not fit in registers)
+        const int c_beg = h * kPlainPerWarp;
+#pragma unroll 1
+        for (int i = 0; i < kPlainPerWarp; ++i) {
+          float v[32];
+          tmem_ld_32x32(tb + (c_beg + i) * 32, v);
+          tmem_wait_ld();
+          if (i + 1 == kPlainPerWarp) release_acc();
+          affine(v, n_blk * N_TILE + (c_beg + i) * 32);
+          emit_f32(v, row0, n_blk * N_TILE + (c_beg + i) * 32);
+        }
+      } else {
+        // SwiGLU: chunk c pairs gate columns c*32.. with up columns n_tile/2 + c*32.. (at most
+        // two chunks per warp, one staging box each)
+        constexpr int kHalf = N_TILE / 2;
+        const int n_mine = glu_end - glu_beg;
+        if (!f32) boxes_free();
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          if (c < n_mine) {
+            const int cc = glu_beg + c;
+            float gt[32], up[32];
+            tmem_ld_32x32(tb + cc * 32, gt);
+            tmem_ld_32x32(tb + kHalf + cc * 32, up);
+            tmem_wait_ld();
+            if (c + 1 == n_mine) release_acc();
+            const int j0 = n_blk * kHalf + cc * 32;
+            affine(gt, j0);
+            affine(up, hN + j0);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) gt[i] = gt[i] / (1.0f + __expf(-gt[i])) * up[i];
+            if (f32) {
+              emit_f32(gt, row0, j0);
+            } else {
+              uint32_t t[16];
+              pack_bf16(gt, t);
+              write_box_bf16(t, c);
             }
           }
+        }
+        if (!f32) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) gt[i] = gt[i] / (1.0f + __expf(-gt[i])) * up[i];
-          emit(gt, row0, j0);
+          for (int c = 0; c < 2; ++c)
+            if (c < n_mine) store_box(stage_out + c * 2048, row0, n_blk * kHalf + (glu_beg + c) * 32);
         }
       }
-      if (++acc == L::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
     // every TMA store issued by this warp has completed before the CTA may exit
     if (lane == 0) bulk_wait_group<0>();
     __syncwarp();
   }
 
+  // Neither CTA frees TMEM or exits while the other may still arrive on its barriers or while the
+  // pair's MMAs may still read its shared memory.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 

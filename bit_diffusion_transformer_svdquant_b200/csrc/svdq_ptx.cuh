@@ -39,6 +39,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Same test with acquire semantics at cluster scope: for barriers that threads of the other CTA of
+// a cluster arrive on (their release must synchronize with this acquire).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Same test, but a thread whose phase is not complete is suspended in hardware for up to
 // `hint_ns` (woken early when the phase completes) instead of returning at once, so a waiting warp
 // does not keep re-issuing barrier operations.
@@ -62,10 +75,15 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // Slow path of mbar_wait_bounded, kept out of line: measured on B200, inlining it made even a wait
 // on an already-completed phase cost ~160 cycles instead of ~16 in the issuing thread.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns, unsigned* status,
-                                            unsigned code, volatile int* abort_flag, bool sleep) {
+                                            unsigned code, volatile int* abort_flag, bool sleep,
+                                            bool cluster_scope = false) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (sleep) {
+    if (cluster_scope) {
+#pragma unroll 1
+      for (int i = 0; i < 32; ++i)
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+    } else if (sleep) {
       if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     } else {
 #pragma unroll 1
@@ -89,6 +107,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort_flag, bool sleep = false) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, limit_ns, status, code, abort_flag, sleep);
+}
+// Bounded wait with cluster-scope acquire (see mbar_try_wait_cluster).
+__device__ __forceinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                                          unsigned* status, unsigned code, volatile int* abort_flag) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, limit_ns, status, code, abort_flag, false, true);
+}
+// Arrive on a barrier given by its shared::cluster address (this CTA's or another CTA's of the
+// cluster), with the instruction's default semantics. Callers order their tensor-memory accesses
+// before it with tcgen05.wait::{ld,st} and tcgen05.fence::before_thread_sync. Measured on B200, the
+// .release.cluster form of this arrive added ~1100 cycles to every round trip it sat on.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // ---------------------------------------------------------------- TMA / bulk copies
@@ -196,6 +227,50 @@ __device__ __forceinline__ void tc_commit_warp(uint32_t bar) {
       "{\n\t.reg .pred e;\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar)
+      : "memory");
+}
+// ---- CTA-pair forms (cta_group::2). Every tcgen05 instruction of a kernel uses one cta_group, so
+// the pair kernel uses these exclusively. One warp in each CTA of the pair allocates (collectively)
+// and frees the same TMEM columns in both CTAs.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// M = 256 across the pair: rows 0..127 of A and D live in the even CTA (shared memory / TMEM at the
+// given addresses), rows 128..255 at the same addresses in the odd CTA; B (N rows, K-major) is split
+// in halves the same way. Issued by the even CTA only (warp-wide call, elect.sync picks the lane).
+__device__ __forceinline__ void mma_nvfp4_pair_warp(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                    uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
+}
+__device__ __forceinline__ void mma_bf16_pair_warp(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Arrive once on the barrier at shared-memory offset `bar` in every CTA of `cta_mask` when all
+// pair MMAs issued so far have completed.
+__device__ __forceinline__ void tc_commit_pair_mc_warp(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}\n" ::"r"(bar),
+      "h"(cta_mask)
       : "memory");
 }
 // 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives lane (base + i).

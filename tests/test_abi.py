@@ -28,9 +28,9 @@ def test_status_strings(L):
 
 
 def test_size_queries(L):
-    # QKV 3072 -> 9216, r = 32 at n_tile 192: codes + 2-atom-padded scales + g_w + inv_lambda + L1s^T + L2^T
+    # QKV 3072 -> 9216, r = 32 at n_tile 256: codes + 2-atom scales + g_w + inv_lambda + L1s^T + L2^T
     nb = L.svdq_weight_bytes(9216, 3072, 32)
-    assert nb >= 9216 * 1536 + 9216 // 192 * 48 * 2 * 512 + 3072 * 4 + 32 * 3072 * 2 + 9216 * 32 * 2
+    assert nb >= 9216 * 1536 + 9216 // 256 * 48 * 2 * 512 + 3072 * 4 + 32 * 3072 * 2 + 9216 * 32 * 2
     assert L.svdq_weight_bytes(9216, 3000, 32) == 0          # K % 256
     assert L.svdq_weight_bytes(9216, 3072, 24) == 0          # r not in {0,16,32,64}
     assert L.svdq_weight_bytes(100, 3072, 32) == 0           # N not a multiple of 128 or 192

@@ -64,13 +64,15 @@ def test_codec_edges_through_kernel1(cuda_device):
 
 
 SMALL_CASES = [
-    # M, K, N, r, bias, swiglu
-    (300, 768, 384, 32, True, False),   # ragged M, two 192-wide tiles
+    # M, K, N, r, bias, swiglu     (tile width: 256 where it divides N, else 192, else 128)
+    (300, 768, 384, 32, True, False),   # ragged M (odd number of 128-row blocks), two 192-wide tiles
     (1, 256, 128, 0, False, False),     # one row, no low-rank branch, 128-wide tile
-    (200, 512, 768, 64, True, True),    # SwiGLU with bias, r = 64
-    (130, 1024, 256, 16, False, True),  # SwiGLU, no bias, 128-wide tile
+    (200, 512, 768, 64, True, True),    # SwiGLU with bias, r = 64, three 256-wide tiles
+    (130, 1024, 256, 16, False, True),  # SwiGLU, no bias, one 256-wide tile
     (513, 256, 192, 32, False, False),  # a ragged fifth m-tile, K = one k-step
     (1000, 2048, 1152, 32, True, False),
+    (257, 512, 640, 32, True, True),    # SwiGLU on 128-wide tiles (double-buffered accumulators)
+    (600, 768, 1024, 32, True, False),  # four 256-wide tiles, ragged M
 ]
 
 
