@@ -389,10 +389,19 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
         s != SVDQ_OK)
       return s;
   }
-  // K split across a cluster of 1, 2 or 4 CTAs so that small M still fills the SMs
+  // K split across a cluster of 1, 2 or 4 CTAs so that small M still fills the SMs. Measured on
+  // B200 (K = 3072, r = 32): pairs beat single CTAs at 36 and 132 row tiles (38 vs 54 us, 52 vs
+  // 60 us) and clusters of 4 (45 and 95 us: fewer clusters of 4 are co-resident). Clusters of 4
+  // only for a handful of row tiles. SVDQ_K1_CLUSTER overrides the size; every CTA keeps whole
+  // 64-column K steps.
   const int m_tiles = act->M_pad / 128;
   int csize = 1;
-  while (csize < 4 && m_tiles * csize < sms && (K / (2 * csize)) % 64 == 0) csize *= 2;
+  if (m_tiles < 2 * sms && (K / 2) % 64 == 0) csize = 2;
+  if (16 * m_tiles <= sms && (K / 4) % 64 == 0) csize = 4;
+  if (const char* env = getenv("SVDQ_K1_CLUSTER"); env != nullptr) {
+    const int c = atoi(env);
+    if ((c == 1 || c == 2 || c == 4) && (K / c) % 64 == 0) csize = c;
+  }
   svdq::QuantActArgs a;
   a.inv_lambda = w->inv_lambda;
   a.g_x = g_x;
