@@ -142,7 +142,8 @@ constexpr int kQTile = 128 * 128;  // 128 rows x 64 bf16
 template <int R>
 struct QuantLayout {
   static constexpr int kL1 = (R * 128 + 1023) / 1024 * 1024;
-  static constexpr int kStage = kQTile + kL1;
+  static constexpr int kLamOff = kQTile + kL1;      // the stage's 64 inverse smoothing factors (fp32)
+  static constexpr int kStage = kQTile + kL1 + 1024;
   static constexpr int kPartOff = kQStages * kStage;
   static constexpr int kPart = R * 128 * 4 + 128 * 4;  // rows padded to R + 1 floats
   static constexpr int kTabOff = kPartOff + kPart;        // 128 fp32: 1 / (dec(s) g_x) per scale code
@@ -225,10 +226,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
       for (int st = 0; st < n_steps; ++st) {
         if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)) break;
         const uint32_t sa = sbase + stage * L::kStage;
-        mbar_arrive_expect_tx(full_bar(stage), kQTile + R * 128);
+        mbar_arrive_expect_tx(full_bar(stage), kQTile + R * 128 + 256);
         const int kx = kbeg + (st << 6);
         tma_load_2d(sa, &tmX, kx, m_tile * 128, full_bar(stage));
         if (R > 0) tma_load_2d(sa + kQTile, &tmL1, kx, 0, full_bar(stage));
+        bulk_load(sa + L::kLamOff, a.inv_lambda + kx, 256, full_bar(stage));
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == kQStages) { stage = 0; phase ^= 1u; }
@@ -275,14 +277,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
       if (!__all_sync(0xffffffffu, got)) break;
       const int kst = kbeg + (st << 6);
       const int k = kst + (b << 4);
+      const uint8_t* tile = smem + stage * L::kStage;
+      // this thread's 16 inverse smoothing factors travelled with the stage (a broadcast read: the
+      // threads of one block index b share them)
       float2 lam[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float4 l = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + k) + j);
+        const float4 l = reinterpret_cast<const float4*>(tile + L::kLamOff)[4 * b + j];
         lam[2 * j] = make_float2(l.x, l.y);
         lam[2 * j + 1] = make_float2(l.z, l.w);
       }
-      const uint8_t* tile = smem + stage * L::kStage;
       uint4 x[2][2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
