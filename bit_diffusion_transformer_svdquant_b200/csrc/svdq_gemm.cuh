@@ -120,6 +120,21 @@ __device__ __forceinline__ uint32_t num_clusters_x() {
 
 constexpr int kGemmThreads = 448;
 
+// Tile order: groups of kGroupPairs row pairs (256 rows each); inside a group the row pairs vary
+// fastest, then the n_tile column blocks. The ~74 pairs in flight then share a few A slabs (a
+// group's A rows, 8 x 256 x K/2 bytes) and sweep B, so A is fetched from DRAM about once even when
+// the output stream evicts older lines from L2.
+constexpr int kGroupPairs = 8;
+__device__ __forceinline__ void tile_coords(int tile, int m_pairs, int n_tiles, int& m_pair, int& n_blk) {
+  const int group_tiles = kGroupPairs * n_tiles;
+  const int g = tile / group_tiles;
+  const int first = g * kGroupPairs;
+  const int gm = m_pairs - first < kGroupPairs ? m_pairs - first : kGroupPairs;
+  const int local = tile - g * group_tiles;
+  m_pair = first + local % gm;
+  n_blk = local / gm;
+}
+
 template <int N_TILE, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     svdq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -189,7 +204,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int sf_row_stride = args.K >> 6;  // 64-wide K atoms per 128-row block
       bool ok = true;
       for (int tile = pair0; ok && tile < args.num_tiles; tile += npairs) {
-        const int m_pair = tile % args.m_pairs, n_blk = tile / args.m_pairs;
+        int m_pair, n_blk;
+        tile_coords(tile, args.m_pairs, args.n_tiles, m_pair, n_blk);
         const int m_blk = 2 * m_pair + static_cast<int>(rank);
         // an odd CTA past the last 128-row block loads zero-filled codes (rows past the tensor) and
         // the last block's scales; none of its rows are stored
@@ -448,7 +464,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive_cluster(cluster_map(acce_bar(acc), 0));
     };
     for (int tile = pair0; tile < args.num_tiles; tile += npairs) {
-      const int m_pair = tile % args.m_pairs, n_blk = tile / args.m_pairs;
+      int m_pair, n_blk;
+      tile_coords(tile, args.m_pairs, args.n_tiles, m_pair, n_blk);
       const int m_blk = 2 * m_pair + static_cast<int>(rank);
       // warp-uniform outcome: tcgen05.ld below is a .sync.aligned warp instruction
       const bool got = mbar_wait_bounded(accf_bar(acc), acc_phase, wait_ns, status, kStatusEpilogue, abort_flag);
