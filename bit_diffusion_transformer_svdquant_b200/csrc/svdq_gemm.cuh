@@ -527,14 +527,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           emit_f32(v, row0, n_blk * N_TILE + (c_beg + i) * 32);
         }
       } else {
-        // SwiGLU: chunk c pairs gate columns c*32.. with up columns n_tile/2 + c*32.. (at most
-        // two chunks per warp, one staging box each)
+        // SwiGLU: output chunk c pairs gate columns c*32.. with up columns n_tile/2 + c*32.. (at
+        // most two chunks per warp, one staging box each)
         constexpr int kHalf = N_TILE / 2;
         const int n_mine = glu_end - glu_beg;
-        if (!f32) boxes_free();
+        if (!f32) {
+          // bf16 out: 16-column halves of the chunks, the next half's gate/up loads in flight while
+          // one is scaled and activated; the accumulator is released after the last load, then
+          // the packed rows are staged and stored
+          boxes_free();
+          const int nh = 2 * n_mine;
+          float g[2][16], u[2][16];
+          auto load_half = [&](int hc, float (&gg)[16], float (&uu)[16]) {
+            const int col = (glu_beg + (hc >> 1)) * 32 + 16 * (hc & 1);
+            tmem_ld_32x16(tb + col, gg);
+            tmem_ld_32x16(tb + kHalf + col, uu);
+          };
+          load_half(0, g[0], u[0]);
+          tmem_wait_ld();
+          constexpr int kMaxHalves = 2 * ((kGluChunks + 1) / 2);
+#pragma unroll
+          for (int hc = 0; hc < kMaxHalves; ++hc) {
+            if (hc < nh) {
+              if (hc + 1 < nh) load_half(hc + 1, g[(hc + 1) & 1], u[(hc + 1) & 1]);
+              else release_acc();
+              const int j0 = n_blk * kHalf + (glu_beg + (hc >> 1)) * 32 + 16 * (hc & 1);
+              float (&gg)[16] = g[hc & 1];
+              float (&uu)[16] = u[hc & 1];
+              // 16 outputs of row `lane` -> two 16-byte chunks of staging box hc / 2 (64B swizzle)
+              uint8_t* box_row = stage_out + (hc >> 1) * 2048 + lane * 64;
+#pragma unroll
+              for (int i = 0; i < 16; i += 8) {
+                float bg[8], bu[8];
+                if (has_bias) {
+                  bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + j0 + i)), bg);
+                  bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + hN + j0 + i)), bu);
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) bg[e] = bu[e] = 0.0f;
+                }
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  const float z0 = fmaf(alpha, gg[i + e], bg[e]), z1 = fmaf(alpha, gg[i + e + 1], bg[e + 1]);
+                  const float y0 = __fdividef(z0, 1.0f + __expf(-z0)) * fmaf(alpha, uu[i + e], bu[e]);
+                  const float y1 = __fdividef(z1, 1.0f + __expf(-z1)) * fmaf(alpha, uu[i + e + 1], bu[e + 1]);
+                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+                  w[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+                const int j = 2 * (hc & 1) + i / 8;
+                *reinterpret_cast<uint4*>(box_row + ((j ^ ((lane >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+              if (hc + 1 < nh) tmem_wait_ld();
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            if (c < n_mine) store_box(stage_out + c * 2048, row0, n_blk * kHalf + (glu_beg + c) * 32);
+        } else {
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          if (c < n_mine) {
+          for (int c = 0; c < n_mine; ++c) {
             const int cc = glu_beg + c;
             float gt[32], up[32];
             tmem_ld_32x32(tb + cc * 32, gt);
@@ -544,21 +596,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const int j0 = n_blk * kHalf + cc * 32;
             affine(gt, j0);
             affine(up, hN + j0);
+            // the same arithmetic as the bf16 path, so that bf16 output = bf16(fp32 output)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) gt[i] = gt[i] / (1.0f + __expf(-gt[i])) * up[i];
-            if (f32) {
-              emit_f32(gt, row0, j0);
-            } else {
-              uint32_t t[16];
-              pack_bf16(gt, t);
-              write_box_bf16(t, c);
-            }
+            for (int i = 0; i < 32; ++i) gt[i] = __fdividef(gt[i], 1.0f + __expf(-gt[i])) * up[i];
+            emit_f32(gt, row0, j0);
           }
-        }
-        if (!f32) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            if (c < n_mine) store_box(stage_out + c * 2048, row0, n_blk * kHalf + (glu_beg + c) * 32);
         }
       }
       if (++acc == kAccBufs) { acc = 0; acc_phase ^= 1u; }
