@@ -146,7 +146,9 @@ def build_layers(wl, dev):
         bias = d["bias"].to(dev) if spec.bias else None
         n_out = spec.N // 2 if spec.swiglu else spec.N
         Y = torch.empty(spec.M, n_out, dtype=torch.bfloat16, device=dev)
-        layers.append({"spec": spec, "X": X, "w": w, "g_x": g_x, "act": act, "bias": bias, "Y": Y})
+        # the layer's dense bf16 weight [N, K] for the cuBLAS baseline
+        layers.append({"spec": spec, "X": X, "w": w, "g_x": g_x, "act": act, "bias": bias, "Y": Y,
+                       "W_dense": d["W"].to(dev)})
         if wl.name.startswith("mlp"):
             svdq.quantize_act(X, w, g_x, act)
             svdq.gemm(act, w, bias, out=Y)
@@ -162,6 +164,28 @@ def run_step(layers, ev=None):
         if ev is not None:
             ev[i].record()
         svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
+
+
+def baseline_step(layers):
+    """The same layer(s) in plain bf16 through cuBLAS: y = X W^T + bias (SiLU(gate) * up for SwiGLU)."""
+    for L in layers:
+        y = torch.nn.functional.linear(L["X"], L["W_dense"], L["bias"])
+        if L["spec"].swiglu:
+            h = y.shape[1] // 2
+            y = torch.nn.functional.silu(y[:, :h]) * y[:, h:]
+
+
+def time_per_step(fn, steps, flush, stream):
+    """Mean CUDA-event time of fn() over `steps` runs, with the L2 flushed (outside the events)
+    before each."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
 
 
 def gpu_arm(args, rank, world, dev):
@@ -234,6 +258,28 @@ def gpu_arm(args, rank, world, dev):
     k1_gbs = [kernel1_bytes(layers[i]["spec"]) / (k1_avg[i] * 1e-3) / 1e9 for i in range(n_l)]
 
     e2e = e2e_arm(args, layers, dev, world)
+
+    # The same step replayed from a CUDA graph (both kernels of every layer captured once), and the
+    # bf16 cuBLAS baseline on the same shapes; same timing protocol, fewer steps.
+    side_steps = max(3, min(K, 50))
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        run_step(layers)
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_step(layers)
+    graph.replay()
+    graph_ms = time_per_step(graph.replay, side_steps, flush, stream)
+    del graph
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out in the graph replays")
+    for _ in range(3):
+        baseline_step(layers)
+    base_ms = time_per_step(lambda: baseline_step(layers), side_steps, flush, stream)
+    graph_ms = max_over_ranks(graph_ms, dev)
+    base_ms = max_over_ranks(base_ms, dev)
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -262,6 +308,14 @@ def gpu_arm(args, rank, world, dev):
                                     " (nominal dense FP4/bf16 ratio)",
                      "algorithmic": f"{gemm_flops / 1e9:.1f} GFLOP per launch (2MNK + 2MrN)"},
         "e2e": e2e,
+        "cuda_graph": {"value": round(world * flops_main / (graph_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                       "ms_per_step": round(graph_ms, 5), "steps": side_steps,
+                       "what": "the timed step (kernel 1 + GEMM of every layer) captured once and replayed"},
+        "bf16_cublas_baseline": {"value": round(world * flops_main / (base_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                                 "ms_per_step": round(base_ms, 5), "steps": side_steps,
+                                 "what": "torch.nn.functional.linear in bf16 (cuBLAS) + bias, SiLU(gate)*up for "
+                                         "SwiGLU, same shapes",
+                                 "speedup_of_this_path": round(base_ms / ms_per_step, 3)},
         "gpu_launches": 2 * n_l * K,
         "clocks": clk.summary(),
         "wall_s_timed_region": round(t_wall, 3),
@@ -352,13 +406,21 @@ def cpu_cores():
 def cpu_baseline(wl, target_s=15.0):
     prepared = oracle_setup(wl)
     rows = choose_rows(prepared, target_s)
+    from oracle import svdquant
     t0 = time.perf_counter()
     oracle_step(prepared, rows)
     dt = time.perf_counter() - t0
+    # the activation-quantization part of the same forward on its own (numpy, vectorised); the
+    # rest is weight decode, the fp64 GEMMs (BLAS) and the epilogue
+    t0 = time.perf_counter()
+    for P in prepared:
+        svdquant.quantize_activations(P["X"][:rows], P["p"]["inv_lambda"], P["g_x"])
+    dq = time.perf_counter() - t0
     flops = sum(2.0 * rows * P["spec"].N * P["spec"].K for P in prepared)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": f"{rows} of {prepared[0]['spec'].M} token rows through every layer of {wl.name} "
-                      f"(fp64 numpy oracle, weights prepared offline), {dt:.1f} s"}
+                      f"(fp64 numpy oracle, weights prepared offline), {dt:.1f} s",
+            "split_s": {"quantize_activations": round(dq, 2), "gemm_and_rest": round(max(dt - dq, 0.0), 2)}}
 
 
 def reference_arm(args):

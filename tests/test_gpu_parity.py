@@ -130,3 +130,28 @@ def test_full_size_workload(cuda_device, spec):
     c.check_weight_codes()
     c.check_act_codes()
     c.check_outputs(samples=3000)
+
+
+def test_cuda_graph_replay(cuda_device):
+    """Both kernels captured in a CUDA graph and replayed give the eager result bit for bit (the
+    library enqueues everything on the caller's stream and allocates nothing per call)."""
+    X, W, b = _rand_layer(300, 768, 512, 32, seed=11, bias=True)
+    c = Case(X, W, b, 32, False, cuda_device)
+    y_eager = c.run_gemm(torch.bfloat16).clone()
+    Y = torch.empty_like(y_eager)
+    side = torch.cuda.Stream(cuda_device)
+    side.wait_stream(torch.cuda.current_stream(cuda_device))
+    with torch.cuda.stream(side):
+        svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
+        svdq.gemm(c.act, c.w, c.bias_d, out=Y)
+    torch.cuda.current_stream(cuda_device).wait_stream(side)
+    Y.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
+        svdq.gemm(c.act, c.w, c.bias_d, out=Y)
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize(cuda_device)
+    assert svdq.device_status() == 0
+    assert torch.equal(Y, y_eager)
