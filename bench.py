@@ -13,6 +13,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -128,17 +129,24 @@ def kernel1_bytes(spec):
 
 
 # ---------------------------------------------------------------------------------------------- GPU arm
-def build_layers(wl, dev):
+def build_layers(wl, dev, lora=0):
     import bit_diffusion_transformer_svdquant_b200 as svdq
-    from bit_diffusion_transformer_svdquant_b200.prepare import prepare_layer
+    from bit_diffusion_transformer_svdquant_b200.prepare import concat_lora, prepare_layer
 
     layers = []
     prev_out = None
-    for spec in wl.layers:
+    for li, spec in enumerate(wl.layers):
         d = synth.make_linear_inputs(spec)
         chained = wl.name.startswith("mlp") and prev_out is not None
         X = prev_out if chained else d["X"].to(dev)
         p = prepare_layer(X, d["W"].to(dev), spec.r, dev)
+        if lora:
+            # a synthetic LoRA adapter on the branch: A ~ N(0, 1/K), B ~ N(0, 0.05^2), seeded
+            g = torch.Generator().manual_seed(1000 + li)
+            A = torch.randn(spec.K, lora, generator=g, dtype=torch.float64) / spec.K ** 0.5
+            B = torch.randn(lora, spec.N, generator=g, dtype=torch.float64) * 0.05
+            p = concat_lora(p, A, B)
+            spec = dataclasses.replace(spec, r=spec.r + lora)
         w = svdq.PackedWeight(p["R"], p["L1s"], p["L2"], p["inv_lambda"], swiglu=spec.swiglu)
         del p
         g_x = svdq.calibrate_act(X, w)
@@ -192,7 +200,7 @@ def gpu_arm(args, rank, world, dev):
     import bit_diffusion_transformer_svdquant_b200 as svdq
 
     wl = synth.WORKLOADS[args.workload]
-    layers = build_layers(wl, dev)
+    layers = build_layers(wl, dev, lora=args.lora)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -290,7 +298,8 @@ def gpu_arm(args, rank, world, dev):
                               + (" swiglu" if L["spec"].swiglu else "") + (" bias" if L["spec"].bias else "")
                               for L in layers],
                    "l2": "flushed between timed steps (256 MB write, outside the events)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "lora_rank": args.lora},
         "tokens_per_s": round(world * tokens / (ms_per_step * 1e-3), 1),
         "tflops_incl_lowrank": round(world * (flops_main + flops_lr) / (ms_per_step * 1e-3) / 1e12, 2),
         "frac_fp4_peak_e2e": round(value / world / fp4_peak, 4),
@@ -456,6 +465,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lora", type=int, default=0,
+                    help="rank of a synthetic LoRA adapter concatenated onto each layer's branch")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -40,3 +40,22 @@ def prepare_layer(X: torch.Tensor, W: torch.Tensor, r: int, device=None) -> dict
     del U, S, Vh, W_hat
     return {"R": R.T.contiguous(), "L1s": L1s.contiguous(), "L2": L2.contiguous(),
             "inv_lambda": inv_lambda.contiguous(), "N": N}
+
+
+@torch.no_grad()
+def concat_lora(prep: dict, A: torch.Tensor, B: torch.Tensor) -> dict:
+    """A LoRA adapter (A [K, r_l], B [r_l, N]) rides on the 16-bit branch: L1s <- [L1s | A],
+    L2 <- [L2 ; B] in bf16, so the packed layer computes X L1s L2 + X A B with the same kernels.
+    The pages only name LoRA support; the concatenation is a reading (the branch reads raw X, as a
+    LoRA adapter does). The total rank must be one the kernels take (16, 32 or 64)."""
+    r0 = 0 if prep["L1s"] is None else prep["L1s"].shape[1]
+    r = r0 + A.shape[1]
+    if r not in (16, 32, 64):
+        raise ValueError(f"rank {r0} + LoRA {A.shape[1]} = {r} is not one of 16, 32, 64")
+    dev = prep["inv_lambda"].device
+    A = A.to(device=dev, dtype=torch.bfloat16)
+    B = B.to(device=dev, dtype=torch.bfloat16)
+    out = dict(prep)
+    out["L1s"] = A.contiguous() if r0 == 0 else torch.cat([prep["L1s"], A], dim=1).contiguous()
+    out["L2"] = B.contiguous() if r0 == 0 else torch.cat([prep["L2"], B], dim=0).contiguous()
+    return out

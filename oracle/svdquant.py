@@ -76,6 +76,21 @@ def prepare_layer(X: np.ndarray, W: np.ndarray, r: int) -> dict:
             "R": np.ascontiguousarray(R_kn.T), "sigma": sigma, "r": r}
 
 
+def add_lora(prep: dict, A: np.ndarray, B: np.ndarray) -> dict:
+    """The layer with a LoRA adapter (A [K, r_l], B [r_l, N], bf16 values) riding on the 16-bit
+    branch: L1s <- [L1s | A], L2 <- [L2 ; B], rank r + r_l. The pages only name LoRA support
+    ("Bringing Nunchaku 4-bit diffusion inference to Diffusers"); the concatenation is a reading:
+    the branch reads raw X, as a LoRA adapter does, so (X [L1s|A]) [L2;B] = X L1s L2 + X A B."""
+    out = dict(prep)
+    K = prep["inv_lambda"].shape[0]
+    L1s = prep["L1s"] if prep["r"] > 0 else np.zeros((K, 0))
+    L2 = prep["L2"] if prep["r"] > 0 else np.zeros((0, B.shape[1]))
+    out["L1s"] = np.concatenate([L1s, np.asarray(A, dtype=np.float64)], axis=1)
+    out["L2"] = np.concatenate([L2, np.asarray(B, dtype=np.float64)], axis=0)
+    out["r"] = prep["r"] + A.shape[1]
+    return out
+
+
 def smooth_activations(X: np.ndarray, inv_lambda: np.ndarray) -> np.ndarray:
     """x_hat = fp32(x * inv_lambda_k); one rounding (bf16 x fp32 is exact in fp64)."""
     return f32(X * inv_lambda[None, :])

@@ -155,3 +155,18 @@ def test_cuda_graph_replay(cuda_device):
     torch.cuda.synchronize(cuda_device)
     assert svdq.device_status() == 0
     assert torch.equal(Y, y_eager)
+
+
+def test_lora_on_the_branch(cuda_device):
+    """A rank-32 LoRA adapter concatenated onto the rank-32 branch (r = 64 through the same
+    kernels) matches the oracle's base layer + X A B."""
+    X, W, b = _rand_layer(300, 768, 512, 32, seed=13, bias=True)
+    rng = np.random.default_rng(17)
+    A = svdquant.bf16_round(rng.standard_normal((768, 32)) / np.sqrt(768))
+    B = svdquant.bf16_round(rng.standard_normal((32, 512)) * 0.05)
+    prep = svdquant.add_lora(svdquant.prepare_layer(X, W, 32), A, B)
+    c = Case(X, W, b, 64, False, cuda_device, prep=prep)
+    c.check_scales()
+    c.check_weight_codes()
+    c.check_act_codes()
+    c.check_outputs()

@@ -136,3 +136,28 @@ def test_quantized_layer_tracks_unquantized_on_tiny_workload():
         y = svdquant.layer_forward(X, p, g_x, svdquant.quantize_weight(p["R"]))
         errs[r] = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert errs[spec.r] < 0.2 and errs[spec.r] <= errs[0] * 1.05
+
+
+def test_lora_on_the_branch_is_additive():
+    """Concatenating a LoRA adapter onto the branch adds exactly X A B to the layer output (the
+    linearity the reading relies on), and r grows by the adapter rank."""
+    rng = np.random.default_rng(7)
+    M, K, N = 24, 64, 48
+    X = svdquant.bf16_round(rng.standard_normal((M, K)))
+    W = svdquant.bf16_round(rng.standard_normal((N, K)) / 8)
+    prep = svdquant.prepare_layer(X, W, 16)
+    A = svdquant.bf16_round(rng.standard_normal((K, 16)) / 8)
+    B = svdquant.bf16_round(rng.standard_normal((16, N)) / 8)
+    lp = svdquant.add_lora(prep, A, B)
+    assert lp["r"] == 32 and lp["L1s"].shape == (K, 32) and lp["L2"].shape == (32, N)
+    g_x = svdquant.calibrate_activation_scale(X, prep["inv_lambda"])
+    wq = svdquant.quantize_weight(prep["R"])
+    base = svdquant.layer_forward(X, prep, g_x, wq)
+    with_lora = svdquant.layer_forward(X, lp, g_x, wq)
+    np.testing.assert_allclose(with_lora, base + (X @ A) @ B, rtol=1e-12, atol=1e-12)
+    # a rank-0 layer plus an adapter is the adapter alone on top of plain W4A4
+    p0 = svdquant.prepare_layer(X, W, 0)
+    wq0 = svdquant.quantize_weight(p0["R"])
+    l0 = svdquant.add_lora(p0, A, B)
+    np.testing.assert_allclose(svdquant.layer_forward(X, l0, g_x, wq0),
+                               svdquant.layer_forward(X, p0, g_x, wq0) + (X @ A) @ B, rtol=1e-12, atol=1e-12)
