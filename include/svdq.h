@@ -16,9 +16,10 @@
  * Two kernels run per layer call:
  *   svdq_quantize_act  -- smoothing x_hat = x * inv_lambda, NVFP4 quantization of x_hat, and the
  *                         down-projection U = X L1s on tensor cores, in one pass over X;
- *   svdq_gemm          -- tcgen05 block-scaled FP4 GEMM (TMA-fed shared-memory ring, TMEM
- *                         accumulators) whose epilogue adds the up-projection U L2 (one bf16 MMA
- *                         into the same accumulator), bias and SwiGLU before one store.
+ *   svdq_gemm          -- tcgen05 block-scaled FP4 GEMM on clusters of two CTAs sharing each
+ *                         256-row tile (TMA-fed shared-memory rings, TMEM accumulators) whose
+ *                         epilogue adds the up-projection U L2 (bf16 MMAs into the same
+ *                         accumulator), bias and SwiGLU before one store.
  *
  * Conventions for every entry point:
  *   - Pointers named as device memory must be device pointers on the current device; the library
@@ -27,8 +28,9 @@
  *   - Work is enqueued on `stream` (a cudaStream_t / CUstream; NULL = legacy default stream) and is
  *     asynchronous; argument checks happen on the host before anything is enqueued, and on a
  *     failed check nothing is enqueued.
- *   - Shapes: K % 256 == 0; N % n_tile == 0 for the n_tile chosen at pack time (one of 192, 128;
- *     SwiGLU needs N even); r in {0, 16, 32, 64}; 1 <= M < 2^24. Device pointers 16-byte aligned.
+ *   - Shapes: K % 256 == 0; N % n_tile == 0 for the n_tile chosen at pack time (256 where it
+ *     divides N, else 192, else 128; SwiGLU needs N even); r in {0, 16, 32, 64}; 1 <= M < 2^24.
+ *     Device pointers 16-byte aligned.
  *     Other shapes return SVDQ_ERR_UNSUPPORTED.
  *   - A device that is not sm_100 returns SVDQ_ERR_UNSUPPORTED. There is no CPU fallback.
  *   - Every device-side wait is bounded; a wait that runs out sets a bit in the library's device
@@ -135,7 +137,8 @@ SVDQ_API svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, 
 
 /* Kernel 2 (per layer call). Y: device [M][N] (or [M][N/2] with SwiGLU) of `out_dtype`,
  * row-major; bias: device bf16 [N] in the original (un-interleaved) column order, NULL unless the
- * epilogue adds one. Rows >= M are not written. */
+ * epilogue adds one. Rows >= M are not written. Everything is enqueued on `stream` and nothing is
+ * allocated, so the call can be captured in a CUDA graph together with svdq_quantize_act. */
 SVDQ_API svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t* bias,
                       svdq_epilogue epi, void* Y, svdq_out_dtype out_dtype, svdq_stream_t stream);
 
