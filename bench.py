@@ -165,9 +165,11 @@ def build_layers(wl, dev, lora=0):
     return layers
 
 
-def run_step(layers, ev=None):
+def run_step(layers, ev=None, dynamic=False):
     import bit_diffusion_transformer_svdquant_b200 as svdq
     for i, L in enumerate(layers):
+        if dynamic:
+            svdq.calibrate_act(L["X"], L["w"], out=L["g_x"])
         svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
         if ev is not None:
             ev[i].record()
@@ -204,8 +206,9 @@ def gpu_arm(args, rank, world, dev):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    dyn = args.dynamic_scale
     for _ in range(args.warmup):
-        run_step(layers)
+        run_step(layers, dynamic=dyn)
     torch.cuda.synchronize(dev)
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out during warm-up")
@@ -217,7 +220,8 @@ def gpu_arm(args, rank, world, dev):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     # kernel-level events: quantize (kernel 1) and GEMM (kernel 2) of every layer
     k_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-              torch.cuda.Event(enable_timing=True)) for _ in range(n_l)] for _ in range(K)]
+              torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(n_l)] for _ in range(K)]
 
     if world > 1:
         torch.distributed.barrier()
@@ -228,7 +232,10 @@ def gpu_arm(args, rank, world, dev):
             flush.zero_()
             starts[s].record(stream)
             for i, L in enumerate(layers):
-                e0, e1, e2 = k_ev[s][i]
+                ec, e0, e1, e2 = k_ev[s][i]
+                ec.record(stream)
+                if dyn:
+                    svdq.calibrate_act(L["X"], L["w"], out=L["g_x"])
                 e0.record(stream)
                 svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
                 e1.record(stream)
@@ -244,8 +251,9 @@ def gpu_arm(args, rank, world, dev):
 
     step_ms = [starts[s].elapsed_time(ends[s]) for s in range(K)]
     total_ms = float(sum(step_ms))
-    k1_ms = [[k_ev[s][i][0].elapsed_time(k_ev[s][i][1]) for s in range(K)] for i in range(n_l)]
-    k2_ms = [[k_ev[s][i][1].elapsed_time(k_ev[s][i][2]) for s in range(K)] for i in range(n_l)]
+    kc_ms = [[k_ev[s][i][0].elapsed_time(k_ev[s][i][1]) for s in range(K)] for i in range(n_l)]
+    k1_ms = [[k_ev[s][i][1].elapsed_time(k_ev[s][i][2]) for s in range(K)] for i in range(n_l)]
+    k2_ms = [[k_ev[s][i][2].elapsed_time(k_ev[s][i][3]) for s in range(K)] for i in range(n_l)]
     total_ms = max_over_ranks(total_ms, dev)
 
     flops_main = sum(layer_flops(L["spec"])[0] for L in layers)
@@ -273,11 +281,11 @@ def gpu_arm(args, rank, world, dev):
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
     with torch.cuda.stream(side):
-        run_step(layers)
+        run_step(layers, dynamic=dyn)
     stream.wait_stream(side)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        run_step(layers)
+        run_step(layers, dynamic=dyn)
     graph.replay()
     graph_ms = time_per_step(graph.replay, side_steps, flush, stream)
     del graph
@@ -299,7 +307,8 @@ def gpu_arm(args, rank, world, dev):
                               for L in layers],
                    "l2": "flushed between timed steps (256 MB write, outside the events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "lora_rank": args.lora},
+                   "lora_rank": args.lora,
+                   "activation_scale": "dynamic (amax pass every step)" if dyn else "static (calibrated once)"},
         "tokens_per_s": round(world * tokens / (ms_per_step * 1e-3), 1),
         "tflops_incl_lowrank": round(world * (flops_main + flops_lr) / (ms_per_step * 1e-3) / 1e12, 2),
         "frac_fp4_peak_e2e": round(value / world / fp4_peak, 4),
@@ -308,6 +317,7 @@ def gpu_arm(args, rank, world, dev):
             "quantize_act_gbs": [round(x, 1) for x in k1_gbs],
             "quantize_act_frac_hbm": [round(x / peaks["hbm_gbs"], 4) for x in k1_gbs],
             "gemm_us": [round(statistics.mean(k2_ms[i]) * 1e3, 2) for i in range(n_l)],
+            **({"dynamic_scale_us": [round(statistics.mean(kc_ms[i]) * 1e3, 2) for i in range(n_l)]} if dyn else {}),
         },
         "roofline": {"bound": "tensor", "kernel": "svdq_gemm_kernel", "achieved": round(achieved, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
@@ -325,7 +335,7 @@ def gpu_arm(args, rank, world, dev):
                                  "what": "torch.nn.functional.linear in bf16 (cuBLAS) + bias, SiLU(gate)*up for "
                                          "SwiGLU, same shapes",
                                  "speedup_of_this_path": round(base_ms / ms_per_step, 3)},
-        "gpu_launches": 2 * n_l * K,
+        "gpu_launches": (4 if dyn else 2) * n_l * K,
         "clocks": clk.summary(),
         "wall_s_timed_region": round(t_wall, 3),
     }
@@ -343,14 +353,14 @@ def e2e_arm(args, layers, dev, world):
     steps = max(3, min(args.steps, 20))
     for _ in range(2):
         layers[0]["X"].copy_(X_host, non_blocking=True)
-        run_step(layers)
+        run_step(layers, dynamic=args.dynamic_scale)
         Y_host.copy_(Y_last, non_blocking=True)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
         layers[0]["X"].copy_(X_host, non_blocking=True)
-        run_step(layers)
+        run_step(layers, dynamic=args.dynamic_scale)
         Y_host.copy_(Y_last, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -465,6 +475,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dynamic-scale", action="store_true",
+                    help="compute the activation scale from each step's X (an extra amax pass)")
     ap.add_argument("--lora", type=int, default=0,
                     help="rank of a synthetic LoRA adapter concatenated onto each layer's branch")
     args = ap.parse_args()

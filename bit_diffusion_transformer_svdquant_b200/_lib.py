@@ -207,8 +207,11 @@ def gemm(act: QuantizedAct, w: PackedWeight, bias: torch.Tensor | None = None, e
     return out
 
 
-def linear(X, w, g_x, bias=None, act=None, out=None, out_dtype=torch.bfloat16):
-    """The whole layer: kernel 1 then kernel 2 on the current stream."""
+def linear(X, w, g_x=None, bias=None, act=None, out=None, out_dtype=torch.bfloat16):
+    """The whole layer: kernel 1 then kernel 2 on the current stream. With g_x None the activation
+    scale is computed from this X first (the dynamic mode: one extra amax pass over X)."""
+    if g_x is None:
+        g_x = calibrate_act(X, w)
     act = QuantizedAct(X.shape[0], w.K, w.r, X.device) if act is None else act
     quantize_act(X, w, g_x, act)
     return gemm(act, w, bias, out=out, out_dtype=out_dtype)

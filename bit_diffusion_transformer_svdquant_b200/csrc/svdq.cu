@@ -359,10 +359,15 @@ svdq_status svdq_calibrate_act(const uint16_t* X, int M, const svdq_weight* w, f
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SVDQ_CUDA(cudaMemsetAsync(g_x_out, 0, 4, st));
-  const size_t n8 = static_cast<size_t>(M) * w->K / 8;
-  svdq::act_amax_kernel<<<grid_for(n8, 256, sms), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(X),
-                                                                 w->inv_lambda, n8, w->K,
-                                                                 reinterpret_cast<unsigned*>(g_x_out));
+  // 128 column chunks of 8 per block along x; rows split over y so that ~16 blocks land per SM
+  const int per_row = w->K / 8;
+  const int gx = (per_row + 127) / 128;
+  int gy = sms * 16 / gx;
+  if (gy > M) gy = M;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  svdq::act_amax_kernel<<<dim3(gx, gy), 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(X), w->inv_lambda,
+                                                      M, w->K, reinterpret_cast<unsigned*>(g_x_out));
   if (svdq_status s = check_launch("act_amax_kernel"); s != SVDQ_OK) return s;
   svdq::finalize_scale_kernel<<<1, 1, 0, st>>>(g_x_out);
   return check_launch("finalize_scale_kernel");

@@ -439,17 +439,41 @@ __global__ void amax_f32_kernel(const float* __restrict__ x, size_t n4, unsigned
   if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_uint(m));
 }
 
-// atomicMax of |x * inv_lambda| over X [M][K] bf16 (8 elements per thread).
+// atomicMax of |x * inv_lambda| over X [M][K] bf16. Thread (blockIdx.x, threadIdx.x) owns the
+// 8-column chunk c of every row blockIdx.y, blockIdx.y + gridDim.y, ...: its 8 inverse smoothing
+// factors stay in registers, and a warp reads 32 consecutive 16-byte chunks of a row (four rows in
+// flight per thread).
 __global__ void act_amax_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ inv_lambda,
-                                size_t n8, int K, unsigned* out) {
+                                int M, int K, unsigned* out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int per_row = K >> 3;
   float m = 0.0f;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int k = static_cast<int>((i * 8) % static_cast<size_t>(K));
-    float v[8];
-    bf16x8_to_f32(ldg_stream(X + i * 8), v);
+  if (c < per_row) {
+    float lam[8];
+    const float4 l0 = __ldg(reinterpret_cast<const float4*>(inv_lambda + 8 * c));
+    const float4 l1 = __ldg(reinterpret_cast<const float4*>(inv_lambda + 8 * c) + 1);
+    lam[0] = l0.x; lam[1] = l0.y; lam[2] = l0.z; lam[3] = l0.w;
+    lam[4] = l1.x; lam[5] = l1.y; lam[6] = l1.z; lam[7] = l1.w;
+    const int G = gridDim.y;
+    const __nv_bfloat16* col = X + 8 * static_cast<size_t>(c);
+    auto take = [&](uint4 raw) {
+      float v[8];
+      bf16x8_to_f32(raw, v);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(__fmul_rn(v[j], __ldg(inv_lambda + k + j))));
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(__fmul_rn(v[j], lam[j])));
+    };
+    int r = blockIdx.y;
+    for (; r + 3 * G < M; r += 4 * G) {
+      const uint4 a0 = ldg_stream(col + static_cast<size_t>(r) * K);
+      const uint4 a1 = ldg_stream(col + static_cast<size_t>(r + G) * K);
+      const uint4 a2 = ldg_stream(col + static_cast<size_t>(r + 2 * G) * K);
+      const uint4 a3 = ldg_stream(col + static_cast<size_t>(r + 3 * G) * K);
+      take(a0);
+      take(a1);
+      take(a2);
+      take(a3);
+    }
+    for (; r < M; r += G) take(ldg_stream(col + static_cast<size_t>(r) * K));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));

@@ -170,3 +170,15 @@ def test_lora_on_the_branch(cuda_device):
     c.check_weight_codes()
     c.check_act_codes()
     c.check_outputs()
+
+
+def test_dynamic_activation_scale(cuda_device):
+    """linear() without g_x computes the scale from the call's own X (the amax pass) and gives
+    exactly the result of the statically calibrated path on the same X; the scale is the oracle's."""
+    X, W, b = _rand_layer(260, 512, 384, 16, seed=21, bias=True)
+    c = Case(X, W, b, 16, False, cuda_device)
+    y_static = svdq.linear(c.Xd, c.w, c.g_x, c.bias_d)
+    y_dynamic = svdq.linear(c.Xd, c.w, None, c.bias_d)
+    torch.cuda.synchronize(cuda_device)
+    assert torch.equal(y_static, y_dynamic)
+    assert float(svdq.calibrate_act(c.Xd, c.w).item()) == c.g_x_ref
