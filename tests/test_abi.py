@@ -101,3 +101,54 @@ def test_bench_max_over_ranks_gloo():
     for p in procs:
         p.join(timeout=60)
     assert res == {0: 2.5, 1: 2.5}
+
+
+def _weight_bytes_for_tile(N, K, r, n_tile):
+    """Bytes of a weight blob laid out for a given tile width (each part 256-byte aligned)."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    atoms = (n_tile + 127) // 128
+    parts = [N * K // 2, N // n_tile * (K // 64) * atoms * 512, 4, K * 4]
+    if r:
+        parts += [r * K * 2, N * r * 2]
+    return sum(up(p) for p in parts)
+
+
+@pytest.mark.parametrize("N,tile", [(512, 256), (9216, 256), (384, 192), (1152, 192), (640, 128), (128, 128)])
+def test_tile_width_choice(L, N, tile):
+    """256 where it divides N, else 192, else 128: visible in the scale-atom count of the blob."""
+    K, r = 512, 32
+    got = L.svdq_weight_bytes(N, K, r)
+    assert got == _weight_bytes_for_tile(N, K, r, tile)
+    for other in (256, 192, 128):
+        # another width that divides N would give a different blob whenever its scale atoms differ
+        if other != tile and N % other == 0 and _weight_bytes_for_tile(N, K, r, other) != \
+                _weight_bytes_for_tile(N, K, r, tile):
+            assert got != _weight_bytes_for_tile(N, K, r, other)
+
+
+def test_tile_width_override(L, monkeypatch):
+    """SVDQ_N_TILE picks another valid width; an invalid one is ignored."""
+    N, K, r = 768, 512, 32  # 768 = 3 x 256 = 4 x 192 = 6 x 128
+    assert L.svdq_weight_bytes(N, K, r) == _weight_bytes_for_tile(N, K, r, 256)
+    monkeypatch.setenv("SVDQ_N_TILE", "128")
+    assert L.svdq_weight_bytes(N, K, r) == _weight_bytes_for_tile(N, K, r, 128)
+    monkeypatch.setenv("SVDQ_N_TILE", "96")
+    assert L.svdq_weight_bytes(N, K, r) == _weight_bytes_for_tile(N, K, r, 256)
+
+
+def test_concat_lora_ranks():
+    """A LoRA adapter extends the branch; the total rank must be one the kernels take."""
+    import torch
+    from bit_diffusion_transformer_svdquant_b200.prepare import concat_lora
+    K, N = 64, 48
+    prep = {"R": torch.zeros(N, K), "L1s": torch.zeros(K, 16, dtype=torch.bfloat16),
+            "L2": torch.zeros(16, N, dtype=torch.bfloat16), "inv_lambda": torch.ones(K)}
+    out = concat_lora(prep, torch.ones(K, 16), torch.full((16, N), 2.0))
+    assert out["L1s"].shape == (K, 32) and out["L2"].shape == (32, N)
+    assert out["L1s"].dtype == torch.bfloat16 and float(out["L1s"][0, 20]) == 1.0 and float(out["L2"][20, 0]) == 2.0
+    assert torch.equal(out["L1s"][:, :16], prep["L1s"])
+    with pytest.raises(ValueError):
+        concat_lora(prep, torch.ones(K, 8), torch.ones(8, N))  # 16 + 8 = 24
+    p0 = dict(prep, L1s=None, L2=None)
+    assert concat_lora(p0, torch.ones(K, 16), torch.ones(16, N))["L1s"].shape == (K, 16)
