@@ -73,6 +73,7 @@ SMALL_CASES = [
     (1000, 2048, 1152, 32, True, False),
     (257, 512, 640, 32, True, True),    # SwiGLU on 128-wide tiles (double-buffered accumulators)
     (600, 768, 1024, 32, True, False),  # four 256-wide tiles, ragged M
+    (170, 512, 384, 32, True, True),    # SwiGLU on 192-wide tiles (2 + 1 output chunks per quadrant)
 ]
 
 
