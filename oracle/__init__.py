@@ -9,6 +9,7 @@ nothing from the product.
 Modules:
   nvfp4     -- E2M1 / E4M3 codecs and the NVFP4 block quantizer.
   svdquant  -- smoothing factors, the low-rank/residual split, and the layer forward.
+  fp8r      -- the row-wise FP8 (W8A8) variant of the same layer (no CUDA path yet).
 
 Pins (what each function is checked against, in ``tests/test_oracle_*.py``):
   codecs            -- the format's printed E2M1 grid and hand-derived tie cases, a closed-form
@@ -21,5 +22,9 @@ Pins (what each function is checked against, in ``tests/test_oracle_*.py``):
                        unrounded residual equals sigma_{r+1}), r=0 giving R = W_hat.
   layer forward     -- brute-force exact-rational triple loop on tiny shapes; r=0 reducing to plain
                        W4A4; SwiGLU closed form and special values.
+  fp8r              -- row quantizer: idempotence with scales held fixed, the amax element landing
+                       on +-448, zero rows, the E4M3 half-ulp error bound, scale invariance under
+                       power-of-two row scaling; layer: exact-rational triple loop, r=0 reducing
+                       to plain W8A8.
 No function here is left without a pin.
 """
