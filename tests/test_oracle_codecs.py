@@ -107,6 +107,42 @@ def test_dense_fp32_sweep_against_closed_form(fmt, hi_bits, stride):
         assert np.array_equal(dec(enc(v)), closed(v)), (fmt, hex(lo))
 
 
+# Every rounding decision of E2M1 lies in [2^-3, 2^3) (below 0.25 all round to zero, above 6 all
+# saturate) and every decision of E4M3 in [2^-11, 2^9) (below 2^-10 zero, above 464 saturation).
+# These windows are checked for every fp32 bit pattern, one binade at a time; the tails are sampled.
+DECISION_WINDOWS = {"e2m1": (-3, 3), "e4m3": (-11, 9)}
+
+
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+def test_every_fp32_in_decision_window(fmt):
+    enc = nvfp4.e2m1_encode if fmt == "e2m1" else nvfp4.e4m3_encode
+    dec = nvfp4.e2m1_decode if fmt == "e2m1" else nvfp4.e4m3_decode
+    closed = e2m1_closed if fmt == "e2m1" else e4m3_closed
+    top = 6.0 if fmt == "e2m1" else 448.0
+    lo_e, hi_e = DECISION_WINDOWS[fmt]
+    mant = np.arange(1 << 23, dtype=np.uint32)
+    for e in range(lo_e, hi_e):
+        bits = mant | np.uint32((e + 127) << 23)
+        v32 = bits.view(np.float32)
+        v = v32.astype(np.float64)
+        codes = enc(v)
+        assert np.array_equal(dec(codes), closed(v)), (fmt, e)
+        if fmt == "e4m3":
+            # torch's cast is not saturating (464 and above become NaN), so it is a second
+            # formulation only below the saturation boundary.
+            fin = v < 464.0
+            ref = torch.from_numpy(v32[fin]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(codes[fin], ref), e
+        neg = enc(-v[::7])
+        sign = np.uint8(0x08 if fmt == "e2m1" else 0x80)
+        assert np.array_equal(neg, codes[::7] | sign), (fmt, e)
+    rng = np.random.default_rng(11)
+    below = rng.integers(0, (lo_e + 127) << 23, 1 << 20, dtype=np.uint32).view(np.float32)
+    above = rng.integers((hi_e + 127) << 23, 0x7F800000, 1 << 20, dtype=np.uint32).view(np.float32)
+    assert np.all(dec(enc(below.astype(np.float64))) == 0.0)
+    assert np.all(dec(enc(above.astype(np.float64))) == top)
+
+
 def test_e4m3_against_torch_float8():
     rng = np.random.default_rng(7)
     v = np.concatenate([
