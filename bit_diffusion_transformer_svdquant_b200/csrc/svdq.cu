@@ -211,6 +211,30 @@ bool shape_ok(int N, int K, int r) {
   return N > 0 && K > 0 && K % 256 == 0 && valid_r(r) && K <= (1 << 20) && N <= (1 << 20) && choose_n_tile(N) > 0;
 }
 
+// The descriptors are plain structs that a caller may also fill by hand: before a launch reads
+// through them, check that they describe a layout that svdq_pack_weight / svdq_act_bind can produce.
+svdq_status check_weight(const svdq_weight* w) {
+  const int t = w->n_tile;
+  if ((t != 256 && t != 192 && t != 128) || w->N <= 0 || w->N % t != 0 || w->N > (1 << 20) || w->K <= 0 ||
+      w->K % 256 != 0 || w->K > (1 << 20) || !valid_r(w->r))
+    return fail(SVDQ_ERR_INVALID_ARG, "weight descriptor N=%d K=%d r=%d n_tile=%d is not one svdq_pack_weight makes",
+                w->N, w->K, w->r, t);
+  if (w->codes == nullptr || w->scales == nullptr || w->g_w == nullptr || w->inv_lambda == nullptr ||
+      (w->r > 0 && (w->L1s_t == nullptr || w->L2_t == nullptr)))
+    return fail(SVDQ_ERR_INVALID_ARG, "weight descriptor has a null buffer");
+  return SVDQ_OK;
+}
+
+svdq_status check_act(const svdq_act* a) {
+  if (a->M < 1 || a->M >= (1 << 24) || a->K <= 0 || a->K % 256 != 0 || a->K > (1 << 20) || !valid_r(a->r) ||
+      a->M_pad != (a->M + 127) / 128 * 128)
+    return fail(SVDQ_ERR_INVALID_ARG, "act descriptor M=%d M_pad=%d K=%d r=%d is not one svdq_act_bind makes", a->M,
+                a->M_pad, a->K, a->r);
+  if (a->codes == nullptr || a->scales == nullptr || a->alpha == nullptr || (a->r > 0 && a->U == nullptr))
+    return fail(SVDQ_ERR_INVALID_ARG, "act descriptor has a null buffer");
+  return SVDQ_OK;
+}
+
 int grid_for(size_t work_items, int per_block, int sm_count) {
   size_t blocks = (work_items + per_block - 1) / per_block;
   size_t cap = static_cast<size_t>(sm_count) * 16;
@@ -353,8 +377,10 @@ svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const ui
 
 svdq_status svdq_calibrate_act(const uint16_t* X, int M, const svdq_weight* w, float* g_x_out, svdq_stream_t stream) {
   if (X == nullptr || w == nullptr || g_x_out == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (svdq_status s = check_weight(w); s != SVDQ_OK) return s;
   if (M < 1 || M >= (1 << 24)) return fail(SVDQ_ERR_UNSUPPORTED, "M=%d unsupported", M);
   if (!aligned16(X)) return fail(SVDQ_ERR_UNSUPPORTED, "X must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(g_x_out) & 3u) return fail(SVDQ_ERR_UNSUPPORTED, "g_x_out must be 4-byte aligned");
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -378,7 +404,10 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
   if (X == nullptr || w == nullptr || g_x == nullptr || act == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
   if (act->K != w->K || act->r != w->r)
     return fail(SVDQ_ERR_INVALID_ARG, "act (K=%d r=%d) does not match weight (K=%d r=%d)", act->K, act->r, w->K, w->r);
+  if (svdq_status s = check_weight(w); s != SVDQ_OK) return s;
+  if (svdq_status s = check_act(act); s != SVDQ_OK) return s;
   if (!aligned16(X)) return fail(SVDQ_ERR_UNSUPPORTED, "X must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(g_x) & 3u) return fail(SVDQ_ERR_UNSUPPORTED, "g_x must be 4-byte aligned");
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
   const int K = act->K, r = w->r, M = act->M;
@@ -460,6 +489,8 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
                       svdq_out_dtype out_dtype, svdq_stream_t stream) {
   if (act == nullptr || w == nullptr || Y == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
   if (act->K != w->K || act->r != w->r) return fail(SVDQ_ERR_INVALID_ARG, "act does not match weight");
+  if (svdq_status s = check_weight(w); s != SVDQ_OK) return s;
+  if (svdq_status s = check_act(act); s != SVDQ_OK) return s;
   if (epi < SVDQ_EPI_NONE || epi > SVDQ_EPI_BIAS_SWIGLU) return fail(SVDQ_ERR_INVALID_ARG, "bad epilogue %d", epi);
   if (out_dtype != SVDQ_OUT_BF16 && out_dtype != SVDQ_OUT_F32) return fail(SVDQ_ERR_INVALID_ARG, "bad out dtype");
   const bool has_bias = (epi & 1) != 0, swiglu = (epi & 2) != 0;
@@ -468,8 +499,6 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
   if (!swiglu && w->swiglu_interleaved) return fail(SVDQ_ERR_INVALID_ARG, "weight packed for SwiGLU");
   if (!aligned16(Y) || (bias != nullptr && !aligned16(bias))) return fail(SVDQ_ERR_UNSUPPORTED, "Y / bias alignment");
   const int n_tile = w->n_tile;
-  if ((n_tile != 256 && n_tile != 192 && n_tile != 128) || w->N % n_tile != 0)
-    return fail(SVDQ_ERR_UNSUPPORTED, "bad n_tile");
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
 
@@ -540,6 +569,7 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
 
 svdq_status svdq_export_weight(const svdq_weight* w, uint8_t* codes, uint8_t* scales, svdq_stream_t stream) {
   if (w == nullptr || codes == nullptr || scales == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (svdq_status s = check_weight(w); s != SVDQ_OK) return s;
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
   const size_t total = static_cast<size_t>(w->N) * (w->K / 16);
@@ -551,6 +581,7 @@ svdq_status svdq_export_weight(const svdq_weight* w, uint8_t* codes, uint8_t* sc
 
 svdq_status svdq_export_act(const svdq_act* act, uint8_t* codes, uint8_t* scales, svdq_stream_t stream) {
   if (act == nullptr || codes == nullptr || scales == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (svdq_status s = check_act(act); s != SVDQ_OK) return s;
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
   const size_t total = static_cast<size_t>(act->M) * (act->K / 16);

@@ -59,7 +59,8 @@ typedef void* svdq_stream_t; /* cudaStream_t */
 
 typedef enum {
   SVDQ_OK = 0,
-  SVDQ_ERR_INVALID_ARG = 1, /* null pointer, buffer too small, negative size              */
+  SVDQ_ERR_INVALID_ARG = 1, /* null pointer, buffer too small, negative size, or a          */
+                            /*   descriptor no svdq_pack_weight / svdq_act_bind call makes */
   SVDQ_ERR_UNSUPPORTED = 2, /* shape / alignment / device architecture not supported       */
   SVDQ_ERR_CUDA = 3,        /* a CUDA runtime call failed (message in svdq_last_error)     */
   SVDQ_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out (svdq_device_status)     */
@@ -75,7 +76,8 @@ typedef enum {
 typedef enum { SVDQ_OUT_BF16 = 0, SVDQ_OUT_F32 = 1 } svdq_out_dtype;
 
 /* A packed layer weight. Filled by svdq_pack_weight; every pointer points into the caller's `dst`
- * buffer. Treat as read-only; it may be copied by value. */
+ * buffer. Treat as read-only; it may be copied by value. Every call that takes one first checks
+ * its sizes, n_tile and buffer pointers (SVDQ_ERR_INVALID_ARG before any CUDA call). */
 typedef struct svdq_weight {
   int N, K, r;
   int swiglu_interleaved; /* 1: gate/up rows interleaved per n_tile for the SwiGLU epilogue  */
@@ -91,7 +93,8 @@ typedef struct svdq_weight {
   unsigned long long tmap[2][16]; /* opaque: cached TMA descriptors of codes and L2_t          */
 } svdq_weight;
 
-/* A quantized activation. Bound to caller memory by svdq_act_bind; written by svdq_quantize_act. */
+/* A quantized activation. Bound to caller memory by svdq_act_bind; written by svdq_quantize_act.
+ * Checked like svdq_weight: 1 <= M < 2^24, M_pad as below, K and r valid, buffers non-null. */
 typedef struct svdq_act {
   int M, K, r, M_pad;     /* M_pad = M rounded up to 128                                       */
   void* codes;            /* uint8 [M_pad][K/2] E2M1 codes (rows >= M are zero)                */

@@ -62,6 +62,38 @@ def test_argument_checks_before_any_cuda_call(L):
     assert b"wait limit" in L.svdq_last_error()
 
 
+def _fake_pair(L):
+    """A weight and an act descriptor laid out as the pack / bind calls would, over fake addresses."""
+    base = 1 << 40
+    w = _lib.SvdqWeight(N=512, K=512, r=16, swiglu_interleaved=0, n_tile=256)
+    for i, f in enumerate(("codes", "scales", "g_w", "inv_lambda", "L1s_t", "L2_t")):
+        setattr(w, f, base + (i << 20))
+    act = _lib.SvdqAct()
+    assert L.svdq_act_bind(300, 512, 16, ctypes.c_void_p(base + (64 << 20)), 1 << 30, ctypes.byref(act)) == 0
+    return w, act
+
+
+@pytest.mark.parametrize("field,value", [("n_tile", 100), ("n_tile", 0), ("N", 640), ("K", 500), ("r", 24),
+                                         ("codes", None), ("L2_t", None), ("M_pad", 256), ("M", 0),
+                                         ("alpha", None), ("U", None)])
+def test_descriptor_checks_before_any_cuda_call(L, field, value):
+    """A hand-filled descriptor that no pack / bind call makes is rejected on the host (status 1)."""
+    w, act = _fake_pair(L)
+    p = ctypes.c_void_p(1 << 41)
+    tgt = act if field in ("M_pad", "M", "alpha", "U") else w
+    if field == "K":
+        act.K = value
+    setattr(tgt, field, value)
+    assert L.svdq_gemm(ctypes.byref(act), ctypes.byref(w), None, 0, p, 0, None) == 1, L.svdq_last_error()
+    assert L.svdq_quantize_act(p, ctypes.byref(w), p, ctypes.byref(act), None) == 1, L.svdq_last_error()
+    if tgt is w:
+        assert L.svdq_export_weight(ctypes.byref(w), p, p, None) == 1
+        assert L.svdq_calibrate_act(p, 300, ctypes.byref(w), p, None) == 1
+    else:
+        assert L.svdq_export_act(ctypes.byref(act), p, p, None) == 1
+    assert b"descriptor" in L.svdq_last_error()
+
+
 def test_no_gpu_fails_loudly(L):
     """Valid arguments on a machine without a usable GPU: a CUDA error status, not a fallback."""
     import torch
@@ -70,6 +102,10 @@ def test_no_gpu_fails_loudly(L):
     w = _lib.SvdqWeight()
     p = ctypes.c_void_p(1 << 40)
     st = L.svdq_pack_weight(p, p, p, p, 512, 512, 16, 0, p, 1 << 30, ctypes.byref(w), None)
+    assert st == 3, (st, L.svdq_last_error())
+    # well-formed descriptors get past the host checks and stop at the device query
+    w, act = _fake_pair(L)
+    st = L.svdq_gemm(ctypes.byref(act), ctypes.byref(w), None, 0, p, 0, None)
     assert st == 3, (st, L.svdq_last_error())
 
 
