@@ -33,6 +33,17 @@ class SvdqAct(ctypes.Structure):
                 ("scales", c_void_p), ("U", c_void_p), ("alpha", c_void_p)]
 
 
+class SvdqFp8rWeight(ctypes.Structure):
+    _fields_ = [("N", c_int), ("K", c_int), ("r", c_int), ("swiglu_interleaved", c_int), ("n_tile", c_int),
+                ("reserved0", c_int), ("codes", c_void_p), ("row_scale", c_void_p), ("inv_lambda", c_void_p),
+                ("L1s_t", c_void_p), ("L2_t", c_void_p), ("tmap", c_ulonglong * 32)]
+
+
+class SvdqFp8rAct(ctypes.Structure):
+    _fields_ = [("M", c_int), ("K", c_int), ("r", c_int), ("M_pad", c_int), ("codes", c_void_p),
+                ("row_scale", c_void_p), ("row_rscale", c_void_p), ("U", c_void_p)]
+
+
 class SvdqError(RuntimeError):
     def __init__(self, func: str, status: int, message: str):
         super().__init__(f"{func}: {STATUS_NAMES.get(status, status)}: {message}")
@@ -44,7 +55,17 @@ _lib = None
 
 def _declare(lib):
     W, A = POINTER(SvdqWeight), POINTER(SvdqAct)
+    FW, FA = POINTER(SvdqFp8rWeight), POINTER(SvdqFp8rAct)
     sig = {
+        "svdq_fp8r_weight_bytes": (c_size_t, [c_int, c_int, c_int]),
+        "svdq_fp8r_act_bytes": (c_size_t, [c_int, c_int, c_int]),
+        "svdq_fp8r_pack_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                                          c_void_p, c_size_t, FW, c_void_p]),
+        "svdq_fp8r_act_bind": (c_int, [c_int, c_int, c_int, c_void_p, c_size_t, FA]),
+        "svdq_fp8r_quantize_act": (c_int, [c_void_p, FW, FA, c_void_p]),
+        "svdq_fp8r_gemm": (c_int, [FA, FW, c_void_p, c_int, c_void_p, c_int, c_void_p]),
+        "svdq_fp8r_export_weight": (c_int, [FW, c_void_p, c_void_p, c_void_p]),
+        "svdq_fp8r_export_act": (c_int, [FA, c_void_p, c_void_p, c_void_p]),
         "svdq_weight_bytes": (c_size_t, [c_int, c_int, c_int]),
         "svdq_act_bytes": (c_size_t, [c_int, c_int, c_int]),
         "svdq_pack_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,
@@ -232,6 +253,103 @@ def export_act(act: QuantizedAct):
     with torch.cuda.device(act.device):
         _check("svdq_export_act", lib().svdq_export_act(byref(act.desc), _ptr(codes), _ptr(scales),
                                                         _stream(act.device)))
+    return codes, scales
+
+
+# ---------------------------------------------------------------- row-wise FP8 (W8A8) variant
+
+class Fp8rWeight:
+    """One layer's weight packed for the row-wise FP8 path (E4M3 codes, one fp32 scale per row)."""
+
+    def __init__(self, R: torch.Tensor, L1s: torch.Tensor | None, L2: torch.Tensor | None,
+                 inv_lambda: torch.Tensor, swiglu: bool = False):
+        _need(R, torch.float32, "R", 2)
+        _need(inv_lambda, torch.float32, "inv_lambda", 1)
+        N, K = R.shape
+        r = 0 if L1s is None else L1s.shape[1]
+        if r:
+            _need(L1s, torch.bfloat16, "L1s", 2)
+            _need(L2, torch.bfloat16, "L2", 2)
+            if tuple(L1s.shape) != (K, r) or tuple(L2.shape) != (r, N):
+                raise ValueError("L1s must be [K, r] and L2 [r, N]")
+        nbytes = lib().svdq_fp8r_weight_bytes(N, K, r)
+        if nbytes == 0:
+            raise SvdqError("svdq_fp8r_weight_bytes", 2, f"unsupported shape N={N} K={K} r={r}")
+        self.device = R.device
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=R.device)
+        self.desc = SvdqFp8rWeight()
+        with torch.cuda.device(R.device):
+            _check("svdq_fp8r_pack_weight", lib().svdq_fp8r_pack_weight(
+                _ptr(R), _ptr(L1s) if r else None, _ptr(L2) if r else None, _ptr(inv_lambda), N, K, r,
+                1 if swiglu else 0, _ptr(self.buf), nbytes, byref(self.desc), _stream(R.device)))
+        self.N, self.K, self.r, self.swiglu = N, K, r, swiglu
+
+
+class Fp8rAct:
+    """A row-wise FP8 activation buffer for M rows (codes, row scales, U)."""
+
+    def __init__(self, M: int, K: int, r: int, device):
+        nbytes = lib().svdq_fp8r_act_bytes(M, K, r)
+        if nbytes == 0:
+            raise SvdqError("svdq_fp8r_act_bytes", 2, f"unsupported shape M={M} K={K} r={r}")
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.desc = SvdqFp8rAct()
+        _check("svdq_fp8r_act_bind", lib().svdq_fp8r_act_bind(M, K, r, _ptr(self.buf), nbytes, byref(self.desc)))
+        self.M, self.K, self.r, self.device = M, K, r, self.buf.device
+
+
+def quantize_act_fp8r(X: torch.Tensor, w: Fp8rWeight, act: Fp8rAct) -> Fp8rAct:
+    """Row scales, then smoothing + E4M3 quantization + low-rank down-projection."""
+    _need(X, torch.bfloat16, "X", 2)
+    if X.shape[0] != act.M or X.shape[1] != w.K:
+        raise ValueError("X shape does not match the act buffer / weight")
+    with torch.cuda.device(X.device):
+        _check("svdq_fp8r_quantize_act", lib().svdq_fp8r_quantize_act(_ptr(X), byref(w.desc), byref(act.desc),
+                                                                      _stream(X.device)))
+    return act
+
+
+def gemm_fp8r(act: Fp8rAct, w: Fp8rWeight, bias: torch.Tensor | None = None, epilogue: int | None = None,
+              out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """FP8 GEMM + low-rank up-projection + bias / SwiGLU epilogue."""
+    if epilogue is None:
+        epilogue = (EPI_BIAS if bias is not None else EPI_NONE) | (EPI_SWIGLU if w.swiglu else 0)
+    n_out = w.N // 2 if epilogue & EPI_SWIGLU else w.N
+    if out is None:
+        out = torch.empty(act.M, n_out, dtype=out_dtype, device=act.device)
+    _need(out, out_dtype, "out", 2)
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+    code = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
+    with torch.cuda.device(act.device):
+        _check("svdq_fp8r_gemm", lib().svdq_fp8r_gemm(byref(act.desc), byref(w.desc), _ptr(bias), epilogue,
+                                                      _ptr(out), code, _stream(act.device)))
+    return out
+
+
+def linear_fp8r(X, w: Fp8rWeight, bias=None, act=None, out=None, out_dtype=torch.bfloat16):
+    """The whole row-wise FP8 layer on the current stream (the activation row scales always come
+    from this X)."""
+    act = Fp8rAct(X.shape[0], w.K, w.r, X.device) if act is None else act
+    quantize_act_fp8r(X, w, act)
+    return gemm_fp8r(act, w, bias, out=out, out_dtype=out_dtype)
+
+
+def export_weight_fp8r(w: Fp8rWeight):
+    codes = torch.empty(w.N, w.K, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(w.N, dtype=torch.float32, device=w.device)
+    with torch.cuda.device(w.device):
+        _check("svdq_fp8r_export_weight", lib().svdq_fp8r_export_weight(byref(w.desc), _ptr(codes), _ptr(scales),
+                                                                        _stream(w.device)))
+    return codes, scales
+
+
+def export_act_fp8r(act: Fp8rAct):
+    codes = torch.empty(act.M, act.K, dtype=torch.uint8, device=act.device)
+    scales = torch.empty(act.M, dtype=torch.float32, device=act.device)
+    with torch.cuda.device(act.device):
+        _check("svdq_fp8r_export_act", lib().svdq_fp8r_export_act(byref(act.desc), _ptr(codes), _ptr(scales),
+                                                                  _stream(act.device)))
     return codes, scales
 
 

@@ -12,6 +12,7 @@
 #include <string>
 
 #include "svdq.h"
+#include "svdq_fp8r.cuh"
 #include "svdq_gemm.cuh"
 #include "svdq_ptx.cuh"
 #include "svdq_quant.cuh"
@@ -609,6 +610,424 @@ svdq_status svdq_watchdog_selftest(unsigned long long limit_ns, svdq_stream_t st
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
   svdq::watchdog_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
   return check_launch("watchdog_selftest_kernel");
+}
+
+}  // extern "C"
+
+// ================================================================== row-wise FP8 (W8A8) variant
+namespace {
+
+constexpr int kFp8Stages256 = 6;
+constexpr int kFp8Stages192 = 6;
+constexpr int kFp8Stages128 = 8;
+
+struct Fp8rState {
+  bool ready = false;
+  int max_pairs[3] = {0, 0, 0};  // co-resident CTA pairs of the FP8 GEMM for n_tile 256, 192, 128
+};
+Fp8rState g_fp8r[64];
+
+svdq_status fp8r_max_pairs(const void* fn, int smem, int sms, int* out) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+  cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  int n = 0;
+  SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, fn, &cfg));
+  if (n <= 0) return fail(SVDQ_ERR_CUDA, "FP8 GEMM kernel cannot be resident as CTA pairs");
+  *out = n;
+  return SVDQ_OK;
+}
+
+// The FP8 kernels are set up on the first FP8 call on a device, apart from the NVFP4 set-up (which
+// never depends on them).
+svdq_status fp8r_ready(int* dev_out, int* sm_out) {
+  int dev = 0, sms = 0;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  Fp8rState& st = g_fp8r[dev];
+  if (!st.ready) {
+    using L256 = svdq::fp8r::GemmLayout<256, kFp8Stages256>;
+    using L192 = svdq::fp8r::GemmLayout<192, kFp8Stages192>;
+    using L128 = svdq::fp8r::GemmLayout<128, kFp8Stages128>;
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::gemm_kernel<256, kFp8Stages256>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, L256::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::gemm_kernel<192, kFp8Stages192>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, L192::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::gemm_kernel<128, kFp8Stages128>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, L128::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<0>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<16>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<32>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::QuantLayout<64>::kSmem));
+    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::fp8r::gemm_kernel<256, kFp8Stages256>),
+                                       L256::kSmem, sms, &st.max_pairs[0]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::fp8r::gemm_kernel<192, kFp8Stages192>),
+                                       L192::kSmem, sms, &st.max_pairs[1]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::fp8r::gemm_kernel<128, kFp8Stages128>),
+                                       L128::kSmem, sms, &st.max_pairs[2]);
+        s != SVDQ_OK)
+      return s;
+    st.ready = true;
+  }
+  if (dev_out) *dev_out = dev;
+  if (sm_out) *sm_out = sms;
+  return SVDQ_OK;
+}
+
+struct Fp8rWeightLayout {
+  size_t codes, scales, inv_lambda, l1t, l2t, total;
+};
+Fp8rWeightLayout fp8r_weight_layout(int N, int K, int r) {
+  Fp8rWeightLayout l{};
+  size_t off = 0;
+  l.codes = off;
+  off = align_up(off + static_cast<size_t>(N) * K);
+  l.scales = off;
+  off = align_up(off + static_cast<size_t>(N) * 4);
+  l.inv_lambda = off;
+  off = align_up(off + static_cast<size_t>(K) * 4);
+  l.l1t = off;
+  off = align_up(off + static_cast<size_t>(r) * K * 2);
+  l.l2t = off;
+  off = align_up(off + static_cast<size_t>(N) * r * 2 * 2);  // hi and lo halves
+  l.total = off;
+  return l;
+}
+
+struct Fp8rActLayout {
+  size_t codes, s_x, rs_x, u, total;
+  int M_pad;
+};
+Fp8rActLayout fp8r_act_layout(int M, int K, int r) {
+  Fp8rActLayout l{};
+  l.M_pad = (M + 127) / 128 * 128;
+  size_t off = 0;
+  l.codes = off;
+  off = align_up(off + static_cast<size_t>(l.M_pad) * K);
+  l.s_x = off;
+  off = align_up(off + static_cast<size_t>(l.M_pad) * 4);
+  l.rs_x = off;
+  off = align_up(off + static_cast<size_t>(l.M_pad) * 4);
+  l.u = off;
+  off = align_up(off + static_cast<size_t>(l.M_pad) * r * 2 * 2);  // hi and lo halves
+  l.total = off;
+  return l;
+}
+
+svdq_status check_fp8r_weight(const svdq_fp8r_weight* w) {
+  const int t = w->n_tile;
+  if ((t != 256 && t != 192 && t != 128) || w->N <= 0 || w->N % t != 0 || w->N > (1 << 20) || w->K <= 0 ||
+      w->K % 256 != 0 || w->K > (1 << 20) || !valid_r(w->r))
+    return fail(SVDQ_ERR_INVALID_ARG,
+                "FP8 weight descriptor N=%d K=%d r=%d n_tile=%d is not one svdq_fp8r_pack_weight makes", w->N, w->K,
+                w->r, t);
+  if (w->codes == nullptr || w->row_scale == nullptr || w->inv_lambda == nullptr ||
+      (w->r > 0 && (w->L1s_t == nullptr || w->L2_t == nullptr)))
+    return fail(SVDQ_ERR_INVALID_ARG, "FP8 weight descriptor has a null buffer");
+  return SVDQ_OK;
+}
+
+svdq_status check_fp8r_act(const svdq_fp8r_act* a) {
+  if (a->M < 1 || a->M >= (1 << 24) || a->K <= 0 || a->K % 256 != 0 || a->K > (1 << 20) || !valid_r(a->r) ||
+      a->M_pad != (a->M + 127) / 128 * 128)
+    return fail(SVDQ_ERR_INVALID_ARG,
+                "FP8 act descriptor M=%d M_pad=%d K=%d r=%d is not one svdq_fp8r_act_bind makes", a->M, a->M_pad,
+                a->K, a->r);
+  if (a->codes == nullptr || a->row_scale == nullptr || a->row_rscale == nullptr || (a->r > 0 && a->U == nullptr))
+    return fail(SVDQ_ERR_INVALID_ARG, "FP8 act descriptor has a null buffer");
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t svdq_fp8r_weight_bytes(int N, int K, int r) {
+  if (!shape_ok(N, K, r)) return 0;
+  return fp8r_weight_layout(N, K, r).total;
+}
+
+size_t svdq_fp8r_act_bytes(int M, int K, int r) {
+  if (M < 1 || M >= (1 << 24) || K <= 0 || K % 256 != 0 || K > (1 << 20) || !valid_r(r)) return 0;
+  return fp8r_act_layout(M, K, r).total;
+}
+
+svdq_status svdq_fp8r_act_bind(int M, int K, int r, void* dst, size_t dst_bytes, svdq_fp8r_act* out) {
+  if (out == nullptr || dst == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const size_t need = svdq_fp8r_act_bytes(M, K, r);
+  if (need == 0) return fail(SVDQ_ERR_UNSUPPORTED, "FP8 act shape M=%d K=%d r=%d unsupported", M, K, r);
+  if (dst_bytes < need) return fail(SVDQ_ERR_INVALID_ARG, "FP8 act buffer %zu bytes < %zu", dst_bytes, need);
+  if (reinterpret_cast<uintptr_t>(dst) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "act buffer not 256-byte aligned");
+  const Fp8rActLayout l = fp8r_act_layout(M, K, r);
+  uint8_t* b = static_cast<uint8_t*>(dst);
+  out->M = M;
+  out->K = K;
+  out->r = r;
+  out->M_pad = l.M_pad;
+  out->codes = b + l.codes;
+  out->row_scale = reinterpret_cast<float*>(b + l.s_x);
+  out->row_rscale = reinterpret_cast<float*>(b + l.rs_x);
+  out->U = b + l.u;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_fp8r_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const uint16_t* L2_rn,
+                                  const float* inv_lambda, int N, int K, int r, int swiglu, void* dst,
+                                  size_t dst_bytes, svdq_fp8r_weight* out, svdq_stream_t stream) {
+  if (out == nullptr || R_nk == nullptr || inv_lambda == nullptr || dst == nullptr)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (r > 0 && (L1s_kr == nullptr || L2_rn == nullptr)) return fail(SVDQ_ERR_INVALID_ARG, "null L1s / L2 with r > 0");
+  if (!shape_ok(N, K, r)) return fail(SVDQ_ERR_UNSUPPORTED, "weight shape N=%d K=%d r=%d unsupported", N, K, r);
+  if (!aligned16(R_nk) || !aligned16(inv_lambda) || (r > 0 && (!aligned16(L1s_kr) || !aligned16(L2_rn))))
+    return fail(SVDQ_ERR_UNSUPPORTED, "inputs must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(dst) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "dst not 256-byte aligned");
+  const int n_tile = choose_n_tile(N);
+  const Fp8rWeightLayout l = fp8r_weight_layout(N, K, r);
+  if (dst_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "FP8 weight buffer %zu bytes < %zu", dst_bytes, l.total);
+  int dev, sms;
+  if (svdq_status s = fp8r_ready(&dev, &sms); s != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* b = static_cast<uint8_t*>(dst);
+
+  svdq_fp8r_weight w{};
+  w.N = N;
+  w.K = K;
+  w.r = r;
+  w.swiglu_interleaved = swiglu ? 1 : 0;
+  w.n_tile = n_tile;
+  w.codes = b + l.codes;
+  w.row_scale = reinterpret_cast<float*>(b + l.scales);
+  w.inv_lambda = reinterpret_cast<float*>(b + l.inv_lambda);
+  w.L1s_t = b + l.l1t;
+  w.L2_t = b + l.l2t;
+
+  SVDQ_CUDA(cudaMemcpyAsync(w.inv_lambda, inv_lambda, static_cast<size_t>(K) * 4, cudaMemcpyDeviceToDevice, st));
+  svdq::fp8r::pack_weight_kernel<<<grid_for(static_cast<size_t>(N) * 32, 256, sms), 256, 0, st>>>(
+      R_nk, N, K, n_tile, w.swiglu_interleaved, static_cast<uint8_t*>(w.codes), w.row_scale);
+  if (svdq_status s = check_launch("fp8r::pack_weight_kernel"); s != SVDQ_OK) return s;
+  if (r > 0) {
+    svdq::transpose_l1_kernel<<<grid_for(static_cast<size_t>(K) * r, 256, sms), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(L1s_kr), K, r, static_cast<__nv_bfloat16*>(w.L1s_t));
+    if (svdq_status s = check_launch("transpose_l1_kernel"); s != SVDQ_OK) return s;
+    svdq::fp8r::pack_l2_kernel<<<grid_for(static_cast<size_t>(N) * r, 256, sms), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(L2_rn), w.row_scale, N, r, n_tile, w.swiglu_interleaved,
+        static_cast<__nv_bfloat16*>(w.L2_t));
+    if (svdq_status s = check_launch("fp8r::pack_l2_kernel"); s != SVDQ_OK) return s;
+  }
+  static_assert(sizeof(w.tmap) >= 2 * sizeof(CUtensorMap), "tmap storage");
+  CUtensorMap tmB, tmL2;
+  std::memset(&tmL2, 0, sizeof(tmL2));
+  // each CTA of a GEMM pair stages half of a tile's n_tile rows; one K step is 128 bytes of a row
+  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K, N, K, 128, n_tile / 2,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    // rows 0..N-1: hi halves, rows N..2N-1: lo halves
+    if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, 2 * static_cast<uint64_t>(N),
+                                  static_cast<uint64_t>(r) * 2, r < 32 ? r : 32, n_tile / 2, lr_swizzle(r));
+        s != SVDQ_OK)
+      return s;
+  }
+  std::memcpy(&w.tmap[0][0], &tmB, sizeof(CUtensorMap));
+  std::memcpy(&w.tmap[1][0], &tmL2, sizeof(CUtensorMap));
+  *out = w;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_fp8r_quantize_act(const uint16_t* X, const svdq_fp8r_weight* w, const svdq_fp8r_act* act,
+                                   svdq_stream_t stream) {
+  if (X == nullptr || w == nullptr || act == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (act->K != w->K || act->r != w->r)
+    return fail(SVDQ_ERR_INVALID_ARG, "act (K=%d r=%d) does not match weight (K=%d r=%d)", act->K, act->r, w->K, w->r);
+  if (svdq_status s = check_fp8r_weight(w); s != SVDQ_OK) return s;
+  if (svdq_status s = check_fp8r_act(act); s != SVDQ_OK) return s;
+  if (!aligned16(X)) return fail(SVDQ_ERR_UNSUPPORTED, "X must be 16-byte aligned");
+  int dev, sms;
+  if (svdq_status s = fp8r_ready(&dev, &sms); s != SVDQ_OK) return s;
+  const int K = act->K, r = w->r, M = act->M;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // row scales first: the quantizing pass needs each row's amax before its first code
+  svdq::fp8r::act_row_scale_kernel<<<grid_for(static_cast<size_t>(act->M_pad) * 32, 256, sms), 256, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(X), w->inv_lambda, M, act->M_pad, K, act->row_scale, act->row_rscale);
+  if (svdq_status s = check_launch("fp8r::act_row_scale_kernel"); s != SVDQ_OK) return s;
+  CUtensorMap tmX, tmL1;
+  std::memset(&tmL1, 0, sizeof(tmL1));
+  if (svdq_status s = make_tmap(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(K) * 2, 64, 128,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L1s_t, K, r,
+                                  static_cast<uint64_t>(K) * 2, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+        s != SVDQ_OK)
+      return s;
+  }
+  // K split over a cluster as for the NVFP4 kernel 1 (same structure and stage sizes)
+  const int m_tiles = act->M_pad / 128;
+  int csize = 1;
+  if (m_tiles < 2 * sms && (K / 2) % 64 == 0) csize = 2;
+  if (16 * m_tiles <= sms && (K / 4) % 64 == 0) csize = 4;
+  svdq::fp8r::ActArgs a;
+  a.inv_lambda = w->inv_lambda;
+  a.rs_x = act->row_rscale;
+  a.codes = static_cast<uint8_t*>(act->codes);
+  a.U = static_cast<__nv_bfloat16*>(act->U);
+  a.wait_ns = g_wait_ns.load();
+  a.M = M;
+  a.K = K;
+  a.M_pad = act->M_pad;
+  a.k_per_cta = K / csize;
+
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(m_tiles * csize, 1, 1);
+  cfg.blockDim = dim3(svdq::kQThreads, 1, 1);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaSuccess;
+  switch (r) {
+    case 0:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<0>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<0>, tmX, tmL1, a);
+      break;
+    case 16:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<16>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<16>, tmX, tmL1, a);
+      break;
+    case 32:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<32>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<32>, tmX, tmL1, a);
+      break;
+    case 64:
+      cfg.dynamicSmemBytes = svdq::QuantLayout<64>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<64>, tmX, tmL1, a);
+      break;
+    default: return fail(SVDQ_ERR_UNSUPPORTED, "r=%d unsupported", r);
+  }
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of fp8r::quant_act_kernel failed: %s", cudaGetErrorString(e));
+  return check_launch("fp8r::quant_act_kernel");
+}
+
+svdq_status svdq_fp8r_gemm(const svdq_fp8r_act* act, const svdq_fp8r_weight* w, const uint16_t* bias,
+                           svdq_epilogue epi, void* Y, svdq_out_dtype out_dtype, svdq_stream_t stream) {
+  if (act == nullptr || w == nullptr || Y == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (act->K != w->K || act->r != w->r) return fail(SVDQ_ERR_INVALID_ARG, "act does not match weight");
+  if (svdq_status s = check_fp8r_weight(w); s != SVDQ_OK) return s;
+  if (svdq_status s = check_fp8r_act(act); s != SVDQ_OK) return s;
+  if (epi < SVDQ_EPI_NONE || epi > SVDQ_EPI_BIAS_SWIGLU) return fail(SVDQ_ERR_INVALID_ARG, "bad epilogue %d", epi);
+  if (out_dtype != SVDQ_OUT_BF16 && out_dtype != SVDQ_OUT_F32) return fail(SVDQ_ERR_INVALID_ARG, "bad out dtype");
+  const bool has_bias = (epi & 1) != 0, swiglu = (epi & 2) != 0;
+  if (has_bias && bias == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "epilogue needs a bias");
+  if (swiglu && !w->swiglu_interleaved) return fail(SVDQ_ERR_INVALID_ARG, "SwiGLU needs a weight packed with swiglu=1");
+  if (!swiglu && w->swiglu_interleaved) return fail(SVDQ_ERR_INVALID_ARG, "weight packed for SwiGLU");
+  if (!aligned16(Y) || (bias != nullptr && !aligned16(bias))) return fail(SVDQ_ERR_UNSUPPORTED, "Y / bias alignment");
+  const int n_tile = w->n_tile;
+  int dev, sms;
+  if (svdq_status s = fp8r_ready(&dev, &sms); s != SVDQ_OK) return s;
+
+  const int K = w->K, r = w->r;
+  CUtensorMap tmA, tmU;
+  std::memset(&tmU, 0, sizeof(tmU));
+  if (svdq_status s = make_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, act->codes, K, act->M_pad, K, 128, 128,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act->U, r, 2 * static_cast<uint64_t>(act->M_pad),
+                                  static_cast<uint64_t>(r) * 2, r < 32 ? r : 32, 128, lr_swizzle(r));
+        s != SVDQ_OK)
+      return s;
+  }
+  CUtensorMap tmB, tmL2;  // properly aligned copies of the descriptors cached in the weight
+  std::memcpy(&tmB, &w->tmap[0][0], sizeof(CUtensorMap));
+  std::memcpy(&tmL2, &w->tmap[1][0], sizeof(CUtensorMap));
+
+  svdq::fp8r::GemmArgs g{};
+  g.s_x = act->row_scale;
+  g.s_w = w->row_scale;
+  g.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  g.Y = Y;
+  g.wait_ns = g_wait_ns.load();
+  g.M = act->M;
+  g.M_pad = act->M_pad;
+  g.N = w->N;
+  g.K = K;
+  g.r = r;
+  g.m_tiles = act->M_pad / 128;
+  g.m_pairs = (g.m_tiles + 1) / 2;
+  g.n_tiles = w->N / n_tile;
+  g.k_iters = K / 128;
+  g.num_tiles = g.m_pairs * g.n_tiles;
+  g.ldy = swiglu ? w->N / 2 : w->N;
+  g.out_f32 = out_dtype == SVDQ_OUT_F32 ? 1 : 0;
+  g.epi = static_cast<int>(epi);
+  CUtensorMap tmY;
+  if (svdq_status s = make_tmap(&tmY, g.out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y,
+                                static_cast<uint64_t>(g.ldy), static_cast<uint64_t>(act->M),
+                                static_cast<uint64_t>(g.ldy) * (g.out_f32 ? 4 : 2), 32, 32,
+                                g.out_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+      s != SVDQ_OK)
+    return s;
+  int max_pairs = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    max_pairs = g_fp8r[dev].max_pairs[n_tile == 256 ? 0 : n_tile == 192 ? 1 : 2];
+  }
+  const int pairs = g.num_tiles < max_pairs ? g.num_tiles : max_pairs;
+  const dim3 grid(2 * pairs);  // clusters of 2 CTAs (compiled into the kernel)
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_tile == 256) {
+    svdq::fp8r::gemm_kernel<256, kFp8Stages256>
+        <<<grid, svdq::kGemmThreads, svdq::fp8r::GemmLayout<256, kFp8Stages256>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
+  } else if (n_tile == 192) {
+    svdq::fp8r::gemm_kernel<192, kFp8Stages192>
+        <<<grid, svdq::kGemmThreads, svdq::fp8r::GemmLayout<192, kFp8Stages192>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
+  } else {
+    svdq::fp8r::gemm_kernel<128, kFp8Stages128>
+        <<<grid, svdq::kGemmThreads, svdq::fp8r::GemmLayout<128, kFp8Stages128>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
+  }
+  return check_launch("fp8r::gemm_kernel");
+}
+
+svdq_status svdq_fp8r_export_weight(const svdq_fp8r_weight* w, uint8_t* codes, float* scales, svdq_stream_t stream) {
+  if (w == nullptr || codes == nullptr || scales == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (svdq_status s = check_fp8r_weight(w); s != SVDQ_OK) return s;
+  if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return fail(SVDQ_ERR_UNSUPPORTED, "codes must be 16-byte and scales 4-byte aligned");
+  int dev, sms;
+  if (svdq_status s = fp8r_ready(&dev, &sms); s != SVDQ_OK) return s;
+  const size_t total = static_cast<size_t>(w->N) * (w->K / 16);
+  svdq::fp8r::export_weight_kernel<<<grid_for(total, 256, sms), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w->codes), w->row_scale, w->N, w->K, w->n_tile, w->swiglu_interleaved, codes,
+      scales);
+  return check_launch("fp8r::export_weight_kernel");
+}
+
+svdq_status svdq_fp8r_export_act(const svdq_fp8r_act* act, uint8_t* codes, float* scales, svdq_stream_t stream) {
+  if (act == nullptr || codes == nullptr || scales == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (svdq_status s = check_fp8r_act(act); s != SVDQ_OK) return s;
+  int dev, sms;
+  if (svdq_status s = fp8r_ready(&dev, &sms); s != SVDQ_OK) return s;
+  // the activation codes are already canonical row-major; rows >= M are padding
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SVDQ_CUDA(cudaMemcpyAsync(codes, act->codes, static_cast<size_t>(act->M) * act->K, cudaMemcpyDeviceToDevice, st));
+  SVDQ_CUDA(cudaMemcpyAsync(scales, act->row_scale, static_cast<size_t>(act->M) * 4, cudaMemcpyDeviceToDevice, st));
+  return SVDQ_OK;
 }
 
 }  // extern "C"

@@ -165,6 +165,72 @@ SVDQ_API svdq_status svdq_watchdog_selftest(unsigned long long limit_ns, svdq_st
 /* Bounded-wait limit used by the GEMM's barrier waits (default 2 s; 1 ms .. 60 s). */
 SVDQ_API svdq_status svdq_set_wait_limit_ns(unsigned long long ns);
 
+/* ---------------------------------------------------------------------------------------------
+ * Row-wise FP8 (W8A8) variant. "FLUX 3 Image Klein on NVIDIA Blackwell", method 1, names FP8
+ * next to NVFP4, and the Diffusers release notes name row-wise FP8 ("fp8r") weights; no formula
+ * is given. Reading: the layer keeps its SVDQuant structure (smoothing, 16-bit low-rank branch,
+ * quantized residual R); R and the smoothed activations become E4M3 codes with one fp32 scale per
+ * row -- per output row of R, per token of X (from the call's own X):
+ *   s = fp32(amax_row / 448) (1 if amax_row < 2^-100),  q = E4M3_rne_sat(fp32(v * fp32(1 / s))),
+ *   y = s_x[m] s_w[n] sum_k dec(qx) dec(qw) + (X L1s) L2 (+ bias) (-> SwiGLU).
+ * Same conventions as the NVFP4 calls above (caller-owned memory, stream-ordered, no allocation,
+ * host checks before any work, SVDQ_ERR_INVALID_ARG for descriptors no pack / bind call makes).
+ * Not yet run on a B200: these calls have no GPU parity record. */
+typedef struct svdq_fp8r_weight {
+  int N, K, r;
+  int swiglu_interleaved; /* 1: gate/up rows interleaved per n_tile, as for svdq_weight         */
+  int n_tile;             /* GEMM tile width along N (256 / 192 / 128, as for svdq_weight)      */
+  int reserved0;
+  void* codes;            /* uint8 [N][K] E4M3 codes, rows in GEMM order                         */
+  float* row_scale;       /* device fp32 [N] s_w per GEMM row                                    */
+  float* inv_lambda;      /* device fp32 [K] smoothing reciprocals                               */
+  void* L1s_t;            /* bf16 [r][K] = (diag(lambda)^-1 L1)^T                                */
+  void* L2_t;             /* bf16 [2][N][r]: v = fp32(L2^T * fp32(1 / s_w)) per GEMM row, stored */
+                          /*   as hi = bf16(v) (rows 0..N-1) then lo = bf16(v - hi)             */
+  unsigned long long tmap[2][16]; /* opaque: cached TMA descriptors of codes and L2_t            */
+} svdq_fp8r_weight;
+
+typedef struct svdq_fp8r_act {
+  int M, K, r, M_pad;     /* M_pad = M rounded up to 128                                         */
+  void* codes;            /* uint8 [M_pad][K] E4M3 codes (rows >= M are zero)                    */
+  float* row_scale;       /* device fp32 [M_pad] s_x (1 for rows >= M)                           */
+  float* row_rscale;      /* device fp32 [M_pad] fp32(1 / s_x)                                   */
+  void* U;                /* bf16 [2][M_pad][r]: u = fp32(fp32(X L1s) * fp32(1 / s_x)) as hi =    */
+                          /*   bf16(u) then lo = bf16(u - hi)                                    */
+} svdq_fp8r_act;
+
+/* Bytes of device memory an FP8 packed weight / quantized activation needs (0 on bad shapes:
+ * the same shapes as svdq_weight_bytes / svdq_act_bytes). */
+SVDQ_API size_t svdq_fp8r_weight_bytes(int N, int K, int r);
+SVDQ_API size_t svdq_fp8r_act_bytes(int M, int K, int r);
+
+/* Offline pack, arguments as svdq_pack_weight. Computes s_w and the E4M3 codes of every row of
+ * R, and L2^T / s_w as a bf16 hi/lo pair, in the GEMM's row order. */
+SVDQ_API svdq_status svdq_fp8r_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const uint16_t* L2_rn,
+                                  const float* inv_lambda, int N, int K, int r, int swiglu, void* dst,
+                                  size_t dst_bytes, svdq_fp8r_weight* out, svdq_stream_t stream);
+
+/* Host-only: lay an svdq_fp8r_act out over `dst` (device, >= svdq_fp8r_act_bytes, 256-aligned). */
+SVDQ_API svdq_status svdq_fp8r_act_bind(int M, int K, int r, void* dst, size_t dst_bytes, svdq_fp8r_act* out);
+
+/* Per layer call: the row-scale pass over X (s_x, 1/s_x), then the quantizing pass (smoothing,
+ * E4M3 codes, U = X L1s on the tensor cores, stored times 1/s_x). X: device bf16 [M][K]. */
+SVDQ_API svdq_status svdq_fp8r_quantize_act(const uint16_t* X, const svdq_fp8r_weight* w,
+                                   const svdq_fp8r_act* act, svdq_stream_t stream);
+
+/* Per layer call: the FP8 GEMM (tcgen05 kind::f8f6f4) with the branch's up-projection in the
+ * same accumulator and y = s_x s_w acc (+ bias) (-> SwiGLU) in the epilogue. Y, bias, epi and
+ * out_dtype as for svdq_gemm. */
+SVDQ_API svdq_status svdq_fp8r_gemm(const svdq_fp8r_act* act, const svdq_fp8r_weight* w, const uint16_t* bias,
+                           svdq_epilogue epi, void* Y, svdq_out_dtype out_dtype, svdq_stream_t stream);
+
+/* Debug / parity: codes [rows][K] (uint8, 16-byte aligned) and row scales [rows] (fp32) in
+ * canonical form (weight rows in the original order; act rows 0..M-1). */
+SVDQ_API svdq_status svdq_fp8r_export_weight(const svdq_fp8r_weight* w, uint8_t* codes, float* scales,
+                                    svdq_stream_t stream);
+SVDQ_API svdq_status svdq_fp8r_export_act(const svdq_fp8r_act* act, uint8_t* codes, float* scales,
+                                 svdq_stream_t stream);
+
 SVDQ_API const char* svdq_status_str(svdq_status s);
 SVDQ_API const char* svdq_last_error(void);
 SVDQ_API int svdq_abi_version(void);

@@ -188,3 +188,81 @@ def test_concat_lora_ranks():
         concat_lora(prep, torch.ones(K, 8), torch.ones(8, N))  # 16 + 8 = 24
     p0 = dict(prep, L1s=None, L2=None)
     assert concat_lora(p0, torch.ones(K, 16), torch.ones(16, N))["L1s"].shape == (K, 16)
+
+
+# ---------------------------------------------------------------- row-wise FP8 variant (host logic)
+
+def _up(x):
+    return (x + 255) // 256 * 256
+
+
+def test_fp8r_size_queries(L):
+    N, K, r = 9216, 3072, 32
+    want = _up(N * K) + _up(N * 4) + _up(K * 4) + _up(r * K * 2) + _up(2 * N * r * 2)
+    assert L.svdq_fp8r_weight_bytes(N, K, r) == want
+    assert L.svdq_fp8r_weight_bytes(N, 3000, r) == 0
+    assert L.svdq_fp8r_weight_bytes(N, K, 24) == 0
+    assert L.svdq_fp8r_weight_bytes(100, K, r) == 0
+    M = 16896
+    assert L.svdq_fp8r_act_bytes(M, K, r) == _up(M * K) + 2 * _up(M * 4) + _up(2 * M * r * 2)
+    assert L.svdq_fp8r_act_bytes(0, K, r) == 0
+    assert L.svdq_fp8r_act_bytes(M, K, 8) == 0
+
+
+def test_fp8r_act_bind_layout(L):
+    act = _lib.SvdqFp8rAct()
+    base = 1 << 40
+    M, K, r = 300, 512, 16
+    nb = L.svdq_fp8r_act_bytes(M, K, r)
+    assert L.svdq_fp8r_act_bind(M, K, r, ctypes.c_void_p(base), nb, ctypes.byref(act)) == 0
+    assert act.M_pad == 384 and act.codes == base
+    assert act.row_scale - act.codes == 384 * 512
+    assert act.row_rscale - act.row_scale == _up(384 * 4) and act.U - act.row_rscale == _up(384 * 4)
+    assert base + nb - act.U >= 2 * 384 * 16 * 2
+    assert L.svdq_fp8r_act_bind(M, K, r, ctypes.c_void_p(base), nb - 1, ctypes.byref(act)) == 1
+    assert L.svdq_fp8r_act_bind(M, K, r, ctypes.c_void_p(base + 16), nb, ctypes.byref(act)) == 2
+
+
+def _fake_fp8r_pair(L):
+    base = 1 << 40
+    w = _lib.SvdqFp8rWeight(N=512, K=512, r=16, swiglu_interleaved=0, n_tile=256)
+    for i, f in enumerate(("codes", "row_scale", "inv_lambda", "L1s_t", "L2_t")):
+        setattr(w, f, base + (i << 20))
+    act = _lib.SvdqFp8rAct()
+    assert L.svdq_fp8r_act_bind(300, 512, 16, ctypes.c_void_p(base + (64 << 20)), 1 << 30, ctypes.byref(act)) == 0
+    return w, act
+
+
+@pytest.mark.parametrize("field,value", [("n_tile", 96), ("N", 640), ("r", 8), ("codes", None), ("row_scale", None),
+                                         ("L2_t", None), ("M_pad", 512), ("M", -1), ("row_rscale", None), ("U", None)])
+def test_fp8r_descriptor_checks_before_any_cuda_call(L, field, value):
+    w, act = _fake_fp8r_pair(L)
+    p = ctypes.c_void_p(1 << 41)
+    tgt = act if field in ("M_pad", "M", "row_rscale", "U") else w
+    setattr(tgt, field, value)
+    assert L.svdq_fp8r_gemm(ctypes.byref(act), ctypes.byref(w), None, 0, p, 0, None) == 1, L.svdq_last_error()
+    assert L.svdq_fp8r_quantize_act(p, ctypes.byref(w), ctypes.byref(act), None) == 1, L.svdq_last_error()
+    if tgt is w:
+        assert L.svdq_fp8r_export_weight(ctypes.byref(w), p, p, None) == 1
+    else:
+        assert L.svdq_fp8r_export_act(ctypes.byref(act), p, p, None) == 1
+    assert b"descriptor" in L.svdq_last_error()
+
+
+def test_fp8r_argument_checks_and_no_gpu(L):
+    import torch
+    w = _lib.SvdqFp8rWeight()
+    p = ctypes.c_void_p(1 << 40)
+    assert L.svdq_fp8r_pack_weight(None, p, p, p, 512, 512, 16, 0, p, 1 << 30, ctypes.byref(w), None) == 1
+    assert L.svdq_fp8r_pack_weight(p, p, p, p, 500, 512, 16, 0, p, 1 << 30, ctypes.byref(w), None) == 2
+    assert L.svdq_fp8r_pack_weight(p, p, p, p, 512, 512, 16, 0, p, 16, ctypes.byref(w), None) == 1  # dst too small
+    fw, fa = _fake_fp8r_pair(L)
+    fw.swiglu_interleaved = 1
+    assert L.svdq_fp8r_gemm(ctypes.byref(fa), ctypes.byref(fw), None, 0, p, 0, None) == 1      # packed for SwiGLU
+    fw.swiglu_interleaved = 0
+    assert L.svdq_fp8r_gemm(ctypes.byref(fa), ctypes.byref(fw), None, 1, p, 0, None) == 1      # bias missing
+    if torch.cuda.is_available():
+        return
+    st = L.svdq_fp8r_pack_weight(p, p, p, p, 512, 512, 16, 0, p, 1 << 30, ctypes.byref(w), None)
+    assert st == 3, (st, L.svdq_last_error())
+    assert L.svdq_fp8r_gemm(ctypes.byref(fa), ctypes.byref(fw), None, 0, p, 0, None) == 3
