@@ -23,6 +23,19 @@ def test_bf16_round():
     assert svdquant.bf16_round(-3.0) == -3.0
 
 
+def test_bf16_round_against_torch():
+    """torch's fp32 -> bf16 cast (a library routine, round-half-even) on random fp32 values over the
+    normal range and on exact ties (low 16 bits 0x8000, both mantissa parities)."""
+    import torch
+    rng = np.random.default_rng(2)
+    bits = rng.integers(0x00800000, 0x7F000000, 1_000_000, dtype=np.uint32)
+    ties = (bits & np.uint32(0xFFFF0000)) | np.uint32(0x8000)
+    sign = np.where(rng.random(bits.size) < 0.5, np.uint32(0x80000000), np.uint32(0))
+    v32 = np.concatenate([bits | sign, ties | sign]).view(np.float32)
+    ref = torch.from_numpy(v32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(svdquant.bf16_round(v32.astype(np.float64)), ref)
+
+
 def test_smoothing_identity():
     X, W, _ = _small()
     inv, lam = svdquant.smoothing(X, W)
