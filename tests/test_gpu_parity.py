@@ -183,3 +183,22 @@ def test_dynamic_activation_scale(cuda_device):
     torch.cuda.synchronize(cuda_device)
     assert torch.equal(y_static, y_dynamic)
     assert float(svdq.calibrate_act(c.Xd, c.w).item()) == c.g_x_ref
+
+
+@pytest.mark.parametrize("M,K,N,r,swiglu", [(130, 256, 384, 16, False), (200, 512, 512, 32, True)])
+def test_outputs_stay_inside_y(cuda_device, M, K, N, r, swiglu):
+    """Canaries: Y is the first M rows of a larger buffer filled with a marker value; after the GEMM
+    the rows past M still hold the marker (the output TMA stores clip at row M, although the tile
+    computes M_pad rows), and Y equals the output of a call into a fresh tensor."""
+    X, W, _ = _rand_layer(M, K, N, r, seed=M + N, bias=False)
+    c = Case(X, W, None, r, swiglu, cuda_device)
+    n_out = N // 2 if swiglu else N
+    marker = -7680.0  # exact in bf16 and fp32
+    for dt in (torch.bfloat16, torch.float32):
+        big = torch.full((M + 64, n_out), marker, dtype=dt, device=cuda_device)
+        y = svdq.gemm(c.act, c.w, None, out=big[:M], out_dtype=dt)
+        fresh = svdq.gemm(c.act, c.w, None, out_dtype=dt)
+        torch.cuda.synchronize(cuda_device)
+        assert svdq.device_status() == 0
+        assert torch.all(big[M:] == marker)
+        assert torch.equal(y, fresh)
