@@ -266,3 +266,36 @@ def test_fp8r_argument_checks_and_no_gpu(L):
     st = L.svdq_fp8r_pack_weight(p, p, p, p, 512, 512, 16, 0, p, 1 << 30, ctypes.byref(w), None)
     assert st == 3, (st, L.svdq_last_error())
     assert L.svdq_fp8r_gemm(ctypes.byref(fa), ctypes.byref(fw), None, 0, p, 0, None) == 3
+
+
+def test_prepare_layer_matches_oracle_preparation():
+    """The torch offline helper against the oracle's preparation on the same data: identical
+    smoothing reciprocals (bit for bit), the split identity W_hat = diag(lambda') L1s L2 + R to R's
+    fp32 rounding, bf16 branch factors, and r = 0 giving exactly the oracle's R."""
+    import numpy as np
+    import torch
+    from bit_diffusion_transformer_svdquant_b200.prepare import prepare_layer
+    from oracle import svdquant
+    rng = np.random.default_rng(3)
+    M, K, N = 96, 256, 192
+    X = rng.standard_normal((M, K))
+    X[:, rng.choice(K, 4, replace=False)] *= 50
+    X = svdquant.bf16_round(X)
+    X[:, 7] = 0.0                                   # a silent channel: lambda = 1
+    W = svdquant.bf16_round(rng.standard_normal((N, K)) / np.sqrt(K))
+    Xt = torch.from_numpy(X.astype(np.float32)).to(torch.bfloat16)
+    Wt = torch.from_numpy(W.astype(np.float32)).to(torch.bfloat16)
+    ref = svdquant.prepare_layer(X, W, 16)
+    got = prepare_layer(Xt, Wt, 16, torch.device("cpu"))
+    assert np.array_equal(got["inv_lambda"].double().numpy(), ref["inv_lambda"])
+    lam_p = 1.0 / got["inv_lambda"].double().numpy()
+    W_hat = lam_p[:, None] * W.T                                           # [K, N]
+    branch = (lam_p[:, None] * got["L1s"].double().numpy()) @ got["L2"].double().numpy()
+    R = got["R"].double().numpy().T
+    assert np.max(np.abs(W_hat - branch - R)) <= 2.0 ** -23 * np.max(np.abs(W_hat))
+    assert got["L1s"].dtype == torch.bfloat16 and got["L2"].dtype == torch.bfloat16
+    # the branch spans the same rank-16 space as the oracle's (signs of singular vectors may differ)
+    ref_branch = (ref["lam_prime"][:, None] * ref["L1s"]) @ ref["L2"]
+    assert np.max(np.abs(branch - ref_branch)) <= 2e-2 * np.max(np.abs(ref_branch))
+    got0 = prepare_layer(Xt, Wt, 0, torch.device("cpu"))
+    assert np.array_equal(got0["R"].double().numpy(), svdquant.prepare_layer(X, W, 0)["R"])
