@@ -43,3 +43,22 @@ def test_reference_arm_two_ranks_rank0_only():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = _json_lines(r.stdout)
     assert len(lines) == 1 and lines[0]["impl"] == "reference"
+
+
+def test_workload_shapes_and_flop_counts():
+    """The synthetic workloads carry the configured shapes: bench's algorithmic FLOPs per layer
+    (2MNK for the FP4 product, 2Mr(K+N) for the branch) reproduce the per-config GFLOP figures
+    derived from the configuration list (to the 0.1 GFLOP they are quoted at)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from bit_diffusion_transformer_svdquant_b200 import synth
+    want = {"tiny": [(0.134, 0.01)], "qkv_1024": [(260.9, 3.6)], "mlp_1024": [(695.8, 8.2), (347.9, 4.5)],
+            "qkv_2048": [(956.7, 13.3)], "edit_2048": [(1884.4, 26.2), (628.1, 13.1)]}
+    for name, layers in want.items():
+        specs = synth.WORKLOADS[name].layers
+        assert len(specs) == len(layers), name
+        for spec, (fp4, lr) in zip(specs, layers):
+            f, l = bench.layer_flops(spec)
+            digits = 3 if fp4 < 1 else 1
+            assert round(f / 1e9, digits) == fp4, (name, f / 1e9)
+            assert abs(l / 1e9 - lr) <= 0.051, (name, l / 1e9)
