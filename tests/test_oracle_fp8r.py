@@ -102,3 +102,38 @@ def test_r0_is_plain_w8a8():
     sx, qx = fp8r.quantize_activations(X, prep["inv_lambda"])
     plain = (sx[:, None] * nvfp4.e4m3_decode(qx)) @ (wq[0][:, None] * nvfp4.e4m3_decode(wq[1])).T
     np.testing.assert_allclose(fp8r.layer_forward(X, prep, wq), plain, rtol=1e-13, atol=1e-13)
+
+
+def test_branch_hi_lo_scheme_precision():
+    """Precision budget of how the row-wise FP8 kernels carry the branch (a design check, emulated in
+    fp64 with the kernels' explicit roundings): U / s_x and L2^T / s_w as bf16 hi/lo pairs, three
+    products (hi.hi, lo.hi, hi.lo) accumulated with the FP8 product, then times s_x s_w. Its error
+    against the exact (X L1s) L2 stays below 1e-4 of max|y| on an outlier-heavy layer, far inside
+    the 2e-3 bar."""
+    f32 = nvfp4.f32
+    rng = np.random.default_rng(9)
+    M, K, N, r = 256, 1024, 512, 32
+    X = rng.standard_normal((M, K))
+    X[:, rng.choice(K, 10, replace=False)] *= 50
+    X = svdquant.bf16_round(X)
+    W = svdquant.bf16_round(rng.standard_normal((N, K)) / np.sqrt(K))
+    prep = svdquant.prepare_layer(X, W, r)
+    s_w, q_w = fp8r.quantize_weight(prep["R"])
+    s_x, _ = fp8r.quantize_activations(X, prep["inv_lambda"])
+    y = fp8r.layer_forward(X, prep, (s_w, q_w))
+    U = f32(X @ prep["L1s"])                                    # fp32 accumulate on the tensor cores
+    u = f32(U * f32(1.0 / s_x)[:, None])
+    u_hi = svdquant.bf16_round(u)
+    u_lo = svdquant.bf16_round(f32(u - u_hi))
+    v = f32(prep["L2"].T * f32(1.0 / s_w)[:, None])             # [N, r]
+    l_hi = svdquant.bf16_round(v)
+    l_lo = svdquant.bf16_round(f32(v - l_hi))
+    acc = u_hi @ l_hi.T + u_lo @ l_hi.T + u_hi @ l_lo.T
+    branch = f32(s_x[:, None] * s_w[None, :]) * acc
+    exact = (X @ prep["L1s"]) @ prep["L2"]
+    err = np.max(np.abs(branch - exact))
+    assert err <= 1e-4 * np.max(np.abs(y)), err / np.max(np.abs(y))
+    # without L2's lo half (U still hi/lo) the error is ~2^-9 relative to the branch: more than a
+    # hundred times larger, about the size of the whole bar on this layer
+    two = f32(s_x[:, None] * s_w[None, :]) * (u_hi @ l_hi.T + u_lo @ l_hi.T)
+    assert np.max(np.abs(two - exact)) > 100 * err
