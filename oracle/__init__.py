@@ -9,12 +9,15 @@ nothing from the product.
 Modules:
   nvfp4     -- E2M1 / E4M3 codecs and the NVFP4 block quantizer.
   svdquant  -- smoothing factors, the low-rank/residual split, and the layer forward.
-  fp8r      -- the row-wise FP8 (W8A8) variant of the same layer (no CUDA path yet).
+  fp8r      -- the row-wise FP8 (W8A8) variant of the same layer.
 
 Pins (what each function is checked against, in ``tests/test_oracle_*.py``):
-  codecs            -- the format's printed E2M1 grid and hand-derived tie cases, a closed-form
-                       round-half-even formulation over every rounding boundary, and torch's
-                       float8_e4m3fn conversion (a library routine) on a dense sample.
+  codecs            -- the format's printed E2M1 grid and hand-derived tie cases; a closed-form
+                       round-half-even formulation over every rounding boundary and over every
+                       fp32 bit pattern of the window that holds all rounding decisions (the
+                       zero and saturation tails sampled); torch's float8_e4m3fn conversion (a
+                       library routine) over that window below its non-saturating range.
+  bf16 rounding     -- hand-derived ties, and torch's fp32 -> bf16 cast on random values and ties.
   block quantizer   -- quantize/dequantize idempotence with scales held fixed, scale bounds,
                        the amax block landing on the largest E4M3 code, all-zero blocks.
   smoothing         -- the identity X.W = (X.diag(lambda)^-1)(diag(lambda).W) and lambda=1 cases.
