@@ -174,8 +174,7 @@ SVDQ_API svdq_status svdq_set_wait_limit_ns(unsigned long long ns);
  *   s = fp32(amax_row / 448) (1 if amax_row < 2^-100),  q = E4M3_rne_sat(fp32(v * fp32(1 / s))),
  *   y = s_x[m] s_w[n] sum_k dec(qx) dec(qw) + (X L1s) L2 (+ bias) (-> SwiGLU).
  * Same conventions as the NVFP4 calls above (caller-owned memory, stream-ordered, no allocation,
- * host checks before any work, SVDQ_ERR_INVALID_ARG for descriptors no pack / bind call makes).
- * Not yet run on a B200: these calls have no GPU parity record. */
+ * host checks before any work, SVDQ_ERR_INVALID_ARG for descriptors no pack / bind call makes). */
 typedef struct svdq_fp8r_weight {
   int N, K, r;
   int swiglu_interleaved; /* 1: gate/up rows interleaved per n_tile, as for svdq_weight         */

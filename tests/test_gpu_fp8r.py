@@ -4,9 +4,6 @@ Bar, as for the NVFP4 path: row scales and E4M3 codes bit-exact; fp32 outputs wi
 max|y - y_ref| <= 2e-3 * max|y_ref|; bf16 outputs bitwise equal to the bf16 rounding of the fp32
 outputs. The low-rank branch runs as bf16 hi/lo pairs of U / s_x and L2^T / s_w (about 16
 significant bits each), well inside that bar.
-
-These kernels have not yet run on a B200, so the module is skipped: the mark comes off with the
-first run that passes.
 """
 import numpy as np
 import pytest
@@ -17,7 +14,7 @@ from oracle import fp8r, nvfp4, svdquant
 
 from _parity import REL_TOL, to_dev_bf16, to_dev_f32
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="row-wise FP8 kernels not yet run on a B200")]
+pytestmark = pytest.mark.gpu
 
 
 def _rand_layer(M, K, N, r, seed, bias=True, outlier=50.0):
