@@ -107,3 +107,61 @@ def test_fp8r_codec_edges(cuda_device):
     prep_, w, act = _run(X, W, None, 0, False, cuda_device, prep=prep)
     wq = _check_codes(X, prep_, w, act)
     _check_outputs(X, prep_, wq, None, False, w, act, cuda_device)
+
+
+MULTI_TILE = [
+    # more tiles than resident CTA pairs: accumulator double-buffering and the ring / relay
+    # barrier phases carried from one tile to the next
+    (2048, 512, 9216, 32, True, False),   # 256-wide tiles, ~4 per pair
+    (1024, 256, 6144, 16, False, True),   # SwiGLU on 256-wide tiles
+    (1536, 256, 5760, 32, True, False),   # 192-wide tiles (30 column blocks)
+    (1280, 256, 4736, 64, True, True),    # 128-wide tiles (37 column blocks), SwiGLU, r = 64
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,bias,swiglu", MULTI_TILE)
+def test_fp8r_multi_tile(cuda_device, M, K, N, r, bias, swiglu):
+    X, W, b = _rand_layer(M, K, N, r, seed=M + 7 * N, bias=bias)
+    prep, w, act = _run(X, W, b, r, swiglu, cuda_device)
+    wq = _check_codes(X, prep, w, act)
+    _check_outputs(X, prep, wq, b, swiglu, w, act, cuda_device)
+
+
+def _full_layers():
+    from bit_diffusion_transformer_svdquant_b200 import synth
+    return [pytest.param(spec, id=spec.name) for name in ("qkv_2048", "mlp_1024")
+            for spec in synth.WORKLOADS[name].layers]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("spec", _full_layers())
+def test_fp8r_full_size_sampled_rows(cuda_device, spec):
+    """Full-size layers. Token rows are independent in this variant (each has its own scale), so
+    the oracle's values on a row sample are exact: all weight codes and scales, the sampled rows'
+    activation codes and scales, and their outputs within tolerance; bf16 = bf16(fp32) everywhere."""
+    from bit_diffusion_transformer_svdquant_b200 import synth
+    d = synth.make_linear_inputs(spec)
+    X, W = synth.bf16_values(d["X"]), synth.bf16_values(d["W"])
+    b = synth.bf16_values(d["bias"]) if spec.bias else None
+    prep, w, act = _run(X, W, b, spec.r, spec.swiglu, cuda_device)
+    s_w, q_w = fp8r.quantize_weight(prep["R"])
+    c, s = svdq.export_weight_fp8r(w)
+    assert np.array_equal(s.cpu().numpy().astype(np.float64), s_w)
+    assert np.array_equal(c.cpu().numpy(), q_w)
+    M = X.shape[0]
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([rng.choice(M, 200, replace=False), [0, 127, 128, 255, 256, M - 1]]))
+    s_x, q_x = fp8r.quantize_activations(X[rows], prep["inv_lambda"])
+    c, s = svdq.export_act_fp8r(act)
+    assert np.array_equal(s.cpu().numpy()[rows].astype(np.float64), s_x)
+    assert np.array_equal(c.cpu().numpy()[rows], q_x)
+    bias_d = None if b is None else to_dev_bf16(b, cuda_device)
+    y32 = svdq.gemm_fp8r(act, w, bias_d, out_dtype=torch.float32)
+    ybf = svdq.gemm_fp8r(act, w, bias_d, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert svdq.device_status() == 0
+    assert torch.equal(ybf, y32.to(torch.bfloat16))
+    y = y32.cpu().numpy()[rows].astype(np.float64)
+    ref = fp8r.layer_forward(X[rows], prep, (s_w, q_w), b, spec.swiglu)
+    err, scale = np.max(np.abs(y - ref)), np.max(np.abs(ref))
+    assert err <= REL_TOL * scale, f"max err {err:.3e} > {REL_TOL} * {scale:.3e}"
