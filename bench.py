@@ -6,6 +6,10 @@ linear of the workload, on seeded synthetic inputs already resident in HBM. L2 i
 write) between timed steps, outside the timed events. Timing: CUDA events on the launching stream.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl svdq|reference]
+                  [--dynamic-scale] [--lora R] [--no-fp8r] [--no-cpu-baseline]
+
+On one GPU the line also carries the row-wise FP8 variant of the same workload, measured in a
+child process under the same protocol (``fp8r_variant``).
 
 N > 1 runs under torchrun as independent replicas (the layer has no exchange step), weak scaling.
 Prints one JSON line on rank 0.
@@ -17,6 +21,7 @@ import dataclasses
 import json
 import os
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -32,6 +37,7 @@ from bit_diffusion_transformer_svdquant_b200 import synth  # noqa: E402
 METRIC = "W4A4+low-rank linear TFLOPS, % of B200 dense FP4 peak; tokens/s per layer"
 DEFAULT_WORKLOAD = "qkv_2048"
 FP4_PER_BF16 = 4.0   # nominal dense FP4 / dense bf16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0   # nominal dense FP8 / dense bf16 (4.5 / 2.25 PFLOP/s)
 FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch of the GEMM, from the ncu capture summarised in
 # profiles/svdq_gemm_kernel_qkv2048.md, keyed by a hash of the kernel source it was taken on; any
@@ -373,6 +379,114 @@ def e2e_arm(args, layers, dev, world):
             "d2h_bytes_per_step": Y_host.numel() * Y_host.element_size()}
 
 
+# ---------------------------------------------------------------------------------- row-wise FP8 variant
+def fp8r_arm(args, dev):
+    """The row-wise FP8 (W8A8) variant of the same workload under the same timing protocol: per layer
+    the row-scale and quantizing passes (one call) and the FP8 GEMM. Also a sanity figure: the
+    relative error of each layer's bf16 output on its first 256 rows against the unquantized
+    product computed by torch in fp32."""
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+    from bit_diffusion_transformer_svdquant_b200.prepare import prepare_layer
+
+    wl = synth.WORKLOADS[args.workload]
+    layers = []
+    prev_out = None
+    for spec in wl.layers:
+        d = synth.make_linear_inputs(spec)
+        chained = wl.name.startswith("mlp") and prev_out is not None
+        X = prev_out if chained else d["X"].to(dev)
+        W_dense = d["W"].to(dev)
+        p = prepare_layer(X, W_dense, spec.r, dev)
+        w = svdq.Fp8rWeight(p["R"], p["L1s"], p["L2"], p["inv_lambda"], swiglu=spec.swiglu)
+        del p
+        act = svdq.Fp8rAct(spec.M, spec.K, spec.r, dev)
+        bias = d["bias"].to(dev) if spec.bias else None
+        n_out = spec.N // 2 if spec.swiglu else spec.N
+        Y = torch.empty(spec.M, n_out, dtype=torch.bfloat16, device=dev)
+        layers.append({"spec": spec, "X": X, "w": w, "act": act, "bias": bias, "Y": Y, "W_dense": W_dense})
+        if wl.name.startswith("mlp"):
+            svdq.linear_fp8r(X, w, bias, act=act, out=Y)
+            prev_out = Y
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step(ev=None):
+        for i, L in enumerate(layers):
+            if ev is not None:
+                ev[i][0].record(stream)
+            svdq.quantize_act_fp8r(L["X"], L["w"], L["act"])
+            if ev is not None:
+                ev[i][1].record(stream)
+            svdq.gemm_fp8r(L["act"], L["w"], L["bias"], out=L["Y"])
+            if ev is not None:
+                ev[i][2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out during the FP8 warm-up")
+    K, n_l = args.steps, len(layers)
+    se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    kev = [[tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_l)] for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        for s in range(K):
+            flush.zero_()
+            se[s][0].record(stream)
+            step(kev[s])
+            se[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out in the FP8 timed region")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in se)
+    k1 = [statistics.mean(kev[s][i][0].elapsed_time(kev[s][i][1]) for s in range(K)) for i in range(n_l)]
+    k2 = [statistics.mean(kev[s][i][1].elapsed_time(kev[s][i][2]) for s in range(K)) for i in range(n_l)]
+    flops_main = sum(layer_flops(L["spec"])[0] for L in layers)
+    big = max(range(n_l), key=lambda i: layer_flops(layers[i]["spec"])[0])
+    peaks = read_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    achieved = sum(layer_flops(layers[big]["spec"])) / (k2[big] * 1e-3) / 1e12
+    rel = []
+    for L in layers:
+        rows = min(256, L["spec"].M)
+        ref = L["X"][:rows].float() @ L["W_dense"].float().T
+        if L["bias"] is not None:
+            ref = ref + L["bias"].float()
+        if L["spec"].swiglu:
+            h = ref.shape[1] // 2
+            ref = torch.nn.functional.silu(ref[:, :h]) * ref[:, h:]
+        rel.append(round(float((L["Y"][:rows].float() - ref).norm() / ref.norm()), 5))
+    return {"value": round(flops_main / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+            "steps": K, "warmup": args.warmup, "dtype": "fp8 e4m3 row-wise + bf16 low-rank, fp32 acc",
+            "kernels": {"quantize_act_us": [round(x * 1e3, 2) for x in k1],
+                        "gemm_us": [round(x * 1e3, 2) for x in k2]},
+            "roofline": {"bound": "tensor", "kernel": "fp8r::gemm_kernel", "achieved": round(achieved, 1),
+                         "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
+                         "traffic": None,
+                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                                        f"{FP8_PER_BF16} (nominal dense FP8/bf16 ratio)"},
+            "rel_err_vs_unquantized_first_rows": rel,
+            "gpu_launches": 3 * n_l * K, "clocks": clk.summary(),
+            "what": "the same workload through the row-wise FP8 kernels (row-scale pass, quantizing pass, "
+                    "kind::f8f6f4 GEMM), run in a separate process"}
+
+
+def fp8r_side(args):
+    """fp8r_arm in a child process (its own CUDA context and a time limit), so that nothing in it can
+    affect the main measurement; any failure comes back as {"error": ...}."""
+    cmd = [sys.executable, os.path.abspath(__file__), "--fp8r-only", "--workload", args.workload,
+           "--steps", str(max(3, min(args.steps, 50))), "--warmup", "3"]
+    try:
+        r = subprocess.run(cmd, capture_output=True, text=True, timeout=900, cwd=ROOT)
+        lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+        if r.returncode != 0 or not lines:
+            return {"error": f"exit {r.returncode}: {(r.stderr or r.stdout)[-600:]}"}
+        return json.loads(lines[-1])
+    except Exception as e:  # a time-out or an unparsable line: reported, never raised
+        return {"error": repr(e)[:600]}
+
+
 # ---------------------------------------------------------------------------------------------- CPU oracle
 def oracle_setup(wl, rows_hint=64):
     """The oracle's offline preparation for every layer of the workload (not timed)."""
@@ -479,6 +593,8 @@ def main():
                     help="compute the activation scale from each step's X (an extra amax pass)")
     ap.add_argument("--lora", type=int, default=0,
                     help="rank of a synthetic LoRA adapter concatenated onto each layer's branch")
+    ap.add_argument("--no-fp8r", action="store_true", help="skip the row-wise FP8 side measurement")
+    ap.add_argument("--fp8r-only", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -494,12 +610,17 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.fp8r_only:
+        print(json.dumps(fp8r_arm(args, dev)), flush=True)
+        return
     if world > 1:
         from datetime import timedelta
         torch.distributed.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
     try:
         out = gpu_arm(args, rank, world, dev)
         if rank == 0:
+            if world == 1 and not args.no_fp8r:
+                out["fp8r_variant"] = fp8r_side(args)
             if world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
             print(json.dumps(out), flush=True)

@@ -62,3 +62,17 @@ def test_workload_shapes_and_flop_counts():
             digits = 3 if fp4 < 1 else 1
             assert round(f / 1e9, digits) == fp4, (name, f / 1e9)
             assert abs(l / 1e9 - lr) <= 0.051, (name, l / 1e9)
+
+
+def test_fp8r_side_measurement_never_raises():
+    """The row-wise FP8 side measurement runs in a child process; without a usable GPU (or on any
+    failure) it comes back as an error entry and the main line is unaffected."""
+    import argparse
+    import torch
+    if torch.cuda.is_available():
+        import pytest
+        pytest.skip("a GPU is present")
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.fp8r_side(argparse.Namespace(workload="tiny", steps=3))
+    assert set(r) == {"error"} and r["error"].startswith("exit ")
