@@ -8,10 +8,12 @@ Python binding plus the seeded synthetic workloads and an offline weight-prepara
 """
 from ._lib import (EPI_BIAS, EPI_BIAS_SWIGLU, EPI_NONE, EPI_SWIGLU, Fp8rAct, Fp8rWeight, PackedWeight,
                    QuantizedAct, SvdqError, calibrate_act, device_status, export_act, export_act_fp8r,
-                   export_weight, export_weight_fp8r, gemm, gemm_fp8r, linear, linear_fp8r, quantize_act,
+                   export_weight, export_weight_fp8r, gemm, gemm_fp8r, gemm_swiglu_quant, linear, linear_fp8r, mlp,
+                   quantize_act,
                    quantize_act_fp8r, set_wait_limit_ns, watchdog_selftest)
 
 __all__ = ["EPI_BIAS", "EPI_BIAS_SWIGLU", "EPI_NONE", "EPI_SWIGLU", "Fp8rAct", "Fp8rWeight", "PackedWeight",
            "QuantizedAct", "SvdqError", "calibrate_act", "device_status", "export_act", "export_act_fp8r",
-           "export_weight", "export_weight_fp8r", "gemm", "gemm_fp8r", "linear", "linear_fp8r", "quantize_act",
+           "export_weight", "export_weight_fp8r", "gemm", "gemm_fp8r", "gemm_swiglu_quant", "linear", "linear_fp8r",
+           "mlp", "quantize_act",
            "quantize_act_fp8r", "set_wait_limit_ns", "watchdog_selftest"]

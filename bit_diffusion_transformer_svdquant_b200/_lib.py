@@ -66,6 +66,8 @@ def _declare(lib):
         "svdq_fp8r_gemm": (c_int, [FA, FW, c_void_p, c_int, c_void_p, c_int, c_void_p]),
         "svdq_fp8r_export_weight": (c_int, [FW, c_void_p, c_void_p, c_void_p]),
         "svdq_fp8r_export_act": (c_int, [FA, c_void_p, c_void_p, c_void_p]),
+        "svdq_mlp_scratch_bytes": (c_size_t, [c_int, c_int]),
+        "svdq_gemm_swiglu_quant": (c_int, [A, W, c_void_p, W, c_void_p, A, c_void_p, c_size_t, c_void_p, c_void_p]),
         "svdq_weight_bytes": (c_size_t, [c_int, c_int, c_int]),
         "svdq_act_bytes": (c_size_t, [c_int, c_int, c_int]),
         "svdq_pack_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,
@@ -254,6 +256,43 @@ def export_act(act: QuantizedAct):
         _check("svdq_export_act", lib().svdq_export_act(byref(act.desc), _ptr(codes), _ptr(scales),
                                                         _stream(act.device)))
     return codes, scales
+
+
+# ---------------------------------------------------------------- MLP chain with the down layer's
+# kernel 1 fused into the gate/up GEMM's SwiGLU epilogue
+
+def gemm_swiglu_quant(act: QuantizedAct, w: PackedWeight, bias, w_next: PackedWeight, g_x_next: torch.Tensor,
+                      act_next: QuantizedAct, scratch: torch.Tensor | None = None,
+                      h_out: torch.Tensor | None = None) -> QuantizedAct:
+    """The gate/up GEMM with SwiGLU whose epilogue also quantizes h for the next layer (act_next);
+    h itself is stored only into h_out (bf16 [M, N/2]) if given."""
+    if not w.swiglu:
+        raise ValueError("the gate/up weight must be packed with swiglu=True")
+    _need(g_x_next, torch.float32, "g_x_next")
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+    if h_out is not None:
+        _need(h_out, torch.bfloat16, "h_out", 2)
+    need = lib().svdq_mlp_scratch_bytes(act.M, w_next.r)
+    if need == 0:
+        raise SvdqError("svdq_mlp_scratch_bytes", 2, f"unsupported M={act.M} r_next={w_next.r}")
+    if scratch is None:
+        scratch = torch.empty(need, dtype=torch.uint8, device=act.device)
+    with torch.cuda.device(act.device):
+        _check("svdq_gemm_swiglu_quant", lib().svdq_gemm_swiglu_quant(
+            byref(act.desc), byref(w.desc), _ptr(bias), byref(w_next.desc), _ptr(g_x_next), byref(act_next.desc),
+            _ptr(scratch), scratch.numel(), _ptr(h_out), _stream(act.device)))
+    return act_next
+
+
+def mlp(X, w_up: PackedWeight, g_x_up, w_down: PackedWeight, g_x_down, bias_up=None, bias_down=None,
+        out=None, out_dtype=torch.bfloat16):
+    """The MLP chain X -> SwiGLU(X W_up^T + b_up) -> (.) W_down^T + b_down with the down layer's
+    activation quantization done in the gate/up GEMM's epilogue (two GEMM launches, h stays on chip)."""
+    act_up = quantize_act(X, w_up, g_x_up, QuantizedAct(X.shape[0], w_up.K, w_up.r, X.device))
+    act_down = QuantizedAct(X.shape[0], w_down.K, w_down.r, X.device)
+    gemm_swiglu_quant(act_up, w_up, bias_up, w_down, g_x_down, act_down)
+    return gemm(act_down, w_down, bias_down, out=out, out_dtype=out_dtype)
 
 
 # ---------------------------------------------------------------- row-wise FP8 (W8A8) variant

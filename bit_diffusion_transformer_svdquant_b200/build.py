@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(REPO, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libsvdq.so")
 SOURCES = [os.path.join(CSRC, "svdq.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("svdq_ptx.cuh", "svdq_quant.cuh", "svdq_gemm.cuh", "svdq_fp8r.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("svdq_ptx.cuh", "svdq_quant.cuh", "svdq_gemm.cuh", "svdq_fp8r.cuh", "svdq_fused.cuh")] + [
     os.path.join(INCLUDE, "svdq.h")]
 
 NVCC_FLAGS = [

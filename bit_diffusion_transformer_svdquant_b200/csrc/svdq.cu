@@ -13,6 +13,7 @@
 
 #include "svdq.h"
 #include "svdq_fp8r.cuh"
+#include "svdq_fused.cuh"
 #include "svdq_gemm.cuh"
 #include "svdq_ptx.cuh"
 #include "svdq_quant.cuh"
@@ -1031,3 +1032,185 @@ svdq_status svdq_fp8r_export_act(const svdq_fp8r_act* act, uint8_t* codes, float
 }
 
 }  // extern "C"
+
+// ================================================================== MLP chain: kernel 1 fused into SwiGLU
+namespace {
+
+constexpr int kFusedStages = 4;
+constexpr int kMaxSplits = 8;
+
+struct FusedState {
+  bool ready = false;
+  int max_pairs[3] = {0, 0, 0};  // r_next 16, 32, 64
+};
+FusedState g_fused[64];
+
+svdq_status fused_ready(int* dev_out, int* sm_out) {
+  int dev = 0, sms = 0;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  FusedState& st = g_fused[dev];
+  if (!st.ready) {
+    using L16 = svdq::fused::Layout<kFusedStages, 16>;
+    using L32 = svdq::fused::Layout<kFusedStages, 32>;
+    using L64 = svdq::fused::Layout<kFusedStages, 64>;
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 16>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, L16::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 32>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, L32::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 64>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, L64::kSmem));
+    if (svdq_status s = fp8r_max_pairs(
+            reinterpret_cast<const void*>(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 16>), L16::kSmem, sms,
+            &st.max_pairs[0]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = fp8r_max_pairs(
+            reinterpret_cast<const void*>(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 32>), L32::kSmem, sms,
+            &st.max_pairs[1]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = fp8r_max_pairs(
+            reinterpret_cast<const void*>(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 64>), L64::kSmem, sms,
+            &st.max_pairs[2]);
+        s != SVDQ_OK)
+      return s;
+    st.ready = true;
+  }
+  if (dev_out) *dev_out = dev;
+  if (sm_out) *sm_out = sms;
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t svdq_mlp_scratch_bytes(int M, int r_next) {
+  if (M < 1 || M >= (1 << 24) || !(r_next == 16 || r_next == 32 || r_next == 64)) return 0;
+  const size_t m_pad = static_cast<size_t>((M + 127) / 128 * 128);
+  return static_cast<size_t>(kMaxSplits) * m_pad * static_cast<size_t>(r_next) * 4;
+}
+
+svdq_status svdq_gemm_swiglu_quant(const svdq_act* act, const svdq_weight* w, const uint16_t* bias,
+                                   const svdq_weight* w_next, const float* g_x_next, const svdq_act* act_next,
+                                   void* scratch, size_t scratch_bytes, uint16_t* H, svdq_stream_t stream) {
+  if (act == nullptr || w == nullptr || w_next == nullptr || g_x_next == nullptr || act_next == nullptr ||
+      scratch == nullptr)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (act->K != w->K || act->r != w->r) return fail(SVDQ_ERR_INVALID_ARG, "act does not match weight");
+  if (svdq_status s = check_weight(w); s != SVDQ_OK) return s;
+  if (svdq_status s = check_act(act); s != SVDQ_OK) return s;
+  if (svdq_status s = check_weight(w_next); s != SVDQ_OK) return s;
+  if (svdq_status s = check_act(act_next); s != SVDQ_OK) return s;
+  if (!w->swiglu_interleaved || w->n_tile != 256)
+    return fail(SVDQ_ERR_UNSUPPORTED, "the fused MLP path takes a SwiGLU weight packed with 256-wide tiles");
+  if (w_next->swiglu_interleaved) return fail(SVDQ_ERR_INVALID_ARG, "the next layer's weight is packed for SwiGLU");
+  if (w_next->K != w->N / 2) return fail(SVDQ_ERR_INVALID_ARG, "next layer K=%d != N/2=%d", w_next->K, w->N / 2);
+  if (act_next->M != act->M || act_next->K != w_next->K || act_next->r != w_next->r)
+    return fail(SVDQ_ERR_INVALID_ARG, "next act (M=%d K=%d r=%d) does not match", act_next->M, act_next->K,
+                act_next->r);
+  const int r2 = w_next->r;
+  if (r2 != 16 && r2 != 32 && r2 != 64) return fail(SVDQ_ERR_UNSUPPORTED, "next layer rank %d not in 16/32/64", r2);
+  const size_t need = svdq_mlp_scratch_bytes(act->M, r2);
+  if (scratch_bytes < need) return fail(SVDQ_ERR_INVALID_ARG, "scratch %zu bytes < %zu", scratch_bytes, need);
+  if (!aligned16(scratch) || (bias != nullptr && !aligned16(bias)) || (H != nullptr && !aligned16(H)) ||
+      (reinterpret_cast<uintptr_t>(g_x_next) & 3u))
+    return fail(SVDQ_ERR_UNSUPPORTED, "scratch / bias / H / g_x_next alignment");
+  int dev, sms;
+  if (svdq_status s = fused_ready(&dev, &sms); s != SVDQ_OK) return s;
+
+  const int K = w->K, r = w->r, N = w->N, K2 = w_next->K;
+  CUtensorMap tmA, tmU, tmH, tmL1n;
+  std::memset(&tmU, 0, sizeof(tmU));
+  std::memset(&tmH, 0, sizeof(tmH));
+  if (svdq_status s = make_tmap(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, act->codes, K / 2, act->M_pad, K / 2, 128, 128,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act->U, r, 2 * static_cast<uint64_t>(act->M_pad),
+                                  static_cast<uint64_t>(r) * 2, r < 32 ? r : 32, 128, lr_swizzle(r));
+        s != SVDQ_OK)
+      return s;
+  }
+  // the next layer's L1s^T [r2][K2]: per tile, 64-column boxes of this CTA's r2/2 rows
+  if (svdq_status s = make_tmap(&tmL1n, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_next->L1s_t, K2, r2,
+                                static_cast<uint64_t>(K2) * 2, 64, r2 / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (H != nullptr) {
+    // h [M][N/2] bf16, stored from the 128B-swizzled h tile in 64 x 32 boxes
+    if (svdq_status s = make_tmap(&tmH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, static_cast<uint64_t>(N / 2),
+                                  static_cast<uint64_t>(act->M), static_cast<uint64_t>(N / 2) * 2, 64, 32,
+                                  CU_TENSOR_MAP_SWIZZLE_128B);
+        s != SVDQ_OK)
+      return s;
+  }
+  CUtensorMap tmB, tmL2;
+  std::memcpy(&tmB, &w->tmap[0][0], sizeof(CUtensorMap));
+  std::memcpy(&tmL2, &w->tmap[1][0], sizeof(CUtensorMap));
+
+  svdq::fused::Args a{};
+  a.sfa = static_cast<const uint8_t*>(act->scales);
+  a.sfb = static_cast<const uint8_t*>(w->scales);
+  a.alpha = act->alpha;
+  a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  a.wait_ns = g_wait_ns.load();
+  a.M = act->M;
+  a.M_pad = act->M_pad;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.m_tiles = act->M_pad / 128;
+  a.m_pairs = (a.m_tiles + 1) / 2;
+  a.n_tiles = N / 256;
+  a.k_iters = K / 256;
+  a.store_h = H != nullptr ? 1 : 0;
+  a.inv_lambda2 = w_next->inv_lambda;
+  a.g_x2 = g_x_next;
+  a.codes2 = static_cast<uint8_t*>(act_next->codes);
+  a.sf2 = static_cast<uint8_t*>(act_next->scales);
+  a.partials = static_cast<float*>(scratch);
+  a.K2 = K2;
+  int max_pairs = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    max_pairs = g_fused[dev].max_pairs[r2 == 16 ? 0 : r2 == 32 ? 1 : 2];
+  }
+  // column splits: enough units to about fill the resident pairs, each a sweep over n_tiles/splits tiles
+  int splits = max_pairs / a.m_pairs;
+  if (splits < 1) splits = 1;
+  if (splits > kMaxSplits) splits = kMaxSplits;
+  if (splits > a.n_tiles) splits = a.n_tiles;
+  a.splits = splits;
+  a.num_units = a.m_pairs * splits;
+  const int pairs = a.num_units < max_pairs ? a.num_units : max_pairs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(2 * pairs);
+  switch (r2) {
+    case 16:
+      svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 16>
+          <<<grid, svdq::kGemmThreads, svdq::fused::Layout<kFusedStages, 16>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmH,
+                                                                                          tmL1n, a);
+      break;
+    case 32:
+      svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 32>
+          <<<grid, svdq::kGemmThreads, svdq::fused::Layout<kFusedStages, 32>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmH,
+                                                                                          tmL1n, a);
+      break;
+    default:
+      svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 64>
+          <<<grid, svdq::kGemmThreads, svdq::fused::Layout<kFusedStages, 64>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmH,
+                                                                                          tmL1n, a);
+      break;
+  }
+  if (svdq_status s = check_launch("fused::gemm_swiglu_quant_kernel"); s != SVDQ_OK) return s;
+  svdq::fused::finalize_u_kernel<<<grid_for(static_cast<size_t>(act_next->M_pad) * r2, 256, sms), 256, 0, st>>>(
+      static_cast<const float*>(scratch), splits, act->M, act_next->M_pad, r2, g_x_next, w_next->g_w,
+      static_cast<__nv_bfloat16*>(act_next->U), act_next->alpha);
+  return check_launch("fused::finalize_u_kernel");
+}
+
+}  // extern "C"
+

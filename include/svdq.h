@@ -230,6 +230,32 @@ SVDQ_API svdq_status svdq_fp8r_export_weight(const svdq_fp8r_weight* w, uint8_t*
 SVDQ_API svdq_status svdq_fp8r_export_act(const svdq_fp8r_act* act, uint8_t* codes, float* scales,
                                  svdq_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * MLP chain: the down layer's kernel 1 fused into the gate/up GEMM's SwiGLU epilogue. The pages
+ * fuse the branch's down-projection with activation quantization ("Bringing Nunchaku 4-bit
+ * diffusion inference to Diffusers", "SVDQuant deep dive") and fuse SwiGLU into the NVFP4 GEMM
+ * ("FLUX 3 Image Klein on NVIDIA Blackwell", method 1); this call does both for the next layer,
+ * so h = SwiGLU(...) need not cross HBM.
+ *
+ * Scratch bytes for svdq_gemm_swiglu_quant at M tokens and next-layer rank r_next (16/32/64):
+ * the column-split partial sums of U' (fp32). 0 on bad arguments. */
+SVDQ_API size_t svdq_mlp_scratch_bytes(int M, int r_next);
+
+/* One call in place of svdq_gemm (gate/up, SwiGLU) + svdq_quantize_act (down layer):
+ *   act, w, bias  the gate/up layer as for svdq_gemm; w packed with swiglu=1 and n_tile 256
+ *   w_next        the down layer's packed weight (K = w->N / 2, rank 16/32/64)
+ *   g_x_next      device fp32 static activation scale of the down layer (svdq_calibrate_act)
+ *   act_next      the down layer's activation (M = act->M): codes, scales, U and alpha written as
+ *                 svdq_quantize_act would write them from h = bf16(SwiGLU(...)); codes and scales
+ *                 are bit-identical to that path, U agrees to fp32 summation order
+ *   scratch       device, >= svdq_mlp_scratch_bytes(M, r_next), 16-byte aligned
+ *   H             optional device bf16 [M][N/2] that also receives h (NULL: h is not stored)
+ * Not captured by any GPU parity record yet. */
+SVDQ_API svdq_status svdq_gemm_swiglu_quant(const svdq_act* act, const svdq_weight* w, const uint16_t* bias,
+                                   const svdq_weight* w_next, const float* g_x_next,
+                                   const svdq_act* act_next, void* scratch, size_t scratch_bytes,
+                                   uint16_t* H, svdq_stream_t stream);
+
 SVDQ_API const char* svdq_status_str(svdq_status s);
 SVDQ_API const char* svdq_last_error(void);
 SVDQ_API int svdq_abi_version(void);

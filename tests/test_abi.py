@@ -299,3 +299,64 @@ def test_prepare_layer_matches_oracle_preparation():
     assert np.max(np.abs(branch - ref_branch)) <= 2e-2 * np.max(np.abs(ref_branch))
     got0 = prepare_layer(Xt, Wt, 0, torch.device("cpu"))
     assert np.array_equal(got0["R"].double().numpy(), svdquant.prepare_layer(X, W, 0)["R"])
+
+
+# ---------------------------------------------------------------- fused MLP chain (host logic)
+
+def _fake_mlp(L):
+    base = 1 << 40
+
+    def weight(N, K, r, swiglu, n_tile, slot):
+        w = _lib.SvdqWeight(N=N, K=K, r=r, swiglu_interleaved=swiglu, n_tile=n_tile)
+        for i, f in enumerate(("codes", "scales", "g_w", "inv_lambda", "L1s_t", "L2_t")):
+            setattr(w, f, base + (slot << 28) + (i << 20))
+        return w
+
+    def act(M, K, r, slot):
+        a = _lib.SvdqAct()
+        assert L.svdq_act_bind(M, K, r, ctypes.c_void_p(base + (slot << 28)), 1 << 27, ctypes.byref(a)) == 0
+        return a
+
+    return (act(300, 512, 16, 1), weight(1024, 512, 16, 1, 256, 2), weight(384, 512, 32, 0, 192, 3),
+            act(300, 512, 32, 4))
+
+
+def _call_mlp(L, a, w, wn, an, scratch_bytes=1 << 26):
+    p = ctypes.c_void_p(1 << 41)
+    return L.svdq_gemm_swiglu_quant(ctypes.byref(a), ctypes.byref(w), None, ctypes.byref(wn), p, ctypes.byref(an),
+                                    p, scratch_bytes, None, None)
+
+
+def test_mlp_scratch_bytes(L):
+    assert L.svdq_mlp_scratch_bytes(4608, 32) == 8 * 4608 * 32 * 4
+    assert L.svdq_mlp_scratch_bytes(300, 16) == 8 * 384 * 16 * 4
+    assert L.svdq_mlp_scratch_bytes(300, 0) == 0 and L.svdq_mlp_scratch_bytes(0, 32) == 0
+
+
+def test_mlp_fused_argument_checks(L):
+    import torch
+    a, w, wn, an = _fake_mlp(L)
+    w.swiglu_interleaved = 0
+    assert _call_mlp(L, a, w, wn, an) == 2                         # not a SwiGLU weight
+    w.swiglu_interleaved, w.n_tile = 1, 128
+    assert _call_mlp(L, a, w, wn, an) == 2                         # 256-wide tiles only
+    w.n_tile = 256
+    wn.K = 256
+    an.K = 256
+    assert _call_mlp(L, a, w, wn, an) == 1                         # next K != N / 2
+    a, w, wn, an = _fake_mlp(L)
+    wn.swiglu_interleaved = 1
+    assert _call_mlp(L, a, w, wn, an) == 1                         # next layer packed for SwiGLU
+    a, w, wn, an = _fake_mlp(L)
+    assert _call_mlp(L, a, w, wn, an, scratch_bytes=1024) == 1     # scratch too small
+    an2 = _lib.SvdqAct()
+    assert L.svdq_act_bind(256, 512, 32, ctypes.c_void_p(1 << 44), 1 << 27, ctypes.byref(an2)) == 0
+    assert _call_mlp(L, a, w, wn, an2) == 1                        # next act has another M
+    a, w, wn, an = _fake_mlp(L)
+    wn.r = 0
+    an0 = _lib.SvdqAct()
+    assert L.svdq_act_bind(300, 512, 0, ctypes.c_void_p(1 << 44), 1 << 27, ctypes.byref(an0)) == 0
+    assert _call_mlp(L, a, w, wn, an0) == 2                        # next layer needs a branch rank
+    if not torch.cuda.is_available():
+        a, w, wn, an = _fake_mlp(L)
+        assert _call_mlp(L, a, w, wn, an) == 3, L.svdq_last_error()  # well-formed: stops at the device
