@@ -202,3 +202,24 @@ def test_outputs_stay_inside_y(cuda_device, M, K, N, r, swiglu):
         assert svdq.device_status() == 0
         assert torch.all(big[M:] == marker)
         assert torch.equal(y, fresh)
+
+
+MULTI_TILE = [
+    # more tiles than resident CTA pairs on 192- and 128-wide tiles (the full-size workloads all
+    # use 256-wide ones): the 128-wide kernel's double-buffered accumulators and the barrier phases
+    # carried from tile to tile.      pair tiles = ceil(M / 256) x N / n_tile
+    (2048, 512, 4736, 32, True, False),   # 128-wide: 8 x 37 = 296 tiles
+    (1280, 256, 4736, 16, False, True),   # 128-wide SwiGLU: 5 x 37 = 185 tiles
+    (1536, 512, 5760, 32, True, False),   # 192-wide: 6 x 30 = 180 tiles
+    (1100, 256, 5760, 64, True, True),    # 192-wide SwiGLU, r = 64, ragged last row block: 5 x 30
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,bias,swiglu", MULTI_TILE)
+def test_multi_tile_per_pair(cuda_device, M, K, N, r, bias, swiglu):
+    X, W, b = _rand_layer(M, K, N, r, seed=3 * M + N, bias=bias)
+    c = Case(X, W, b, r, swiglu, cuda_device)
+    c.check_scales()
+    c.check_weight_codes()
+    c.check_act_codes()
+    c.check_outputs()
