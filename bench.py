@@ -6,7 +6,7 @@ linear of the workload, on seeded synthetic inputs already resident in HBM. L2 i
 write) between timed steps, outside the timed events. Timing: CUDA events on the launching stream.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl svdq|reference]
-                  [--dynamic-scale] [--lora R] [--no-fp8r] [--no-cpu-baseline]
+                  [--dynamic-scale] [--lora R] [--no-fp8r] [--no-cpu-baseline] [--l2-clean]
 
 On one GPU the line also carries the row-wise FP8 variant of the same workload, measured in a
 child process under the same protocol (``fp8r_variant``).
@@ -191,12 +191,21 @@ def baseline_step(layers):
             y = torch.nn.functional.silu(y[:, :h]) * y[:, h:]
 
 
-def time_per_step(fn, steps, flush, stream):
+def flush_l2(flush, clean=None):
+    """The L2 flush between timed steps (outside the events): write `flush`, 256 MB > L2. With
+    `clean` (a second 256 MB buffer) also read that afterwards, so that the step starts with clean
+    L2 lines rather than up to ~126 MB of dirty flush lines that its first kernel writes back."""
+    flush.zero_()
+    if clean is not None:
+        torch.sum(clean, dtype=torch.int64)
+
+
+def time_per_step(fn, steps, flush, stream, clean=None):
     """Mean CUDA-event time of fn() over `steps` runs, with the L2 flushed (outside the events)
     before each."""
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for e0, e1 in ev:
-        flush.zero_()
+        flush_l2(flush, clean)
         e0.record(stream)
         fn()
         e1.record(stream)
@@ -210,6 +219,7 @@ def gpu_arm(args, rank, world, dev):
     wl = synth.WORKLOADS[args.workload]
     layers = build_layers(wl, dev, lora=args.lora)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if args.l2_clean else None
     stream = torch.cuda.current_stream(dev)
 
     dyn = args.dynamic_scale
@@ -235,7 +245,7 @@ def gpu_arm(args, rank, world, dev):
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         t_wall = time.perf_counter()
         for s in range(K):
-            flush.zero_()
+            flush_l2(flush, clean)
             starts[s].record(stream)
             for i, L in enumerate(layers):
                 ec, e0, e1, e2 = k_ev[s][i]
@@ -293,13 +303,13 @@ def gpu_arm(args, rank, world, dev):
     with torch.cuda.graph(graph):
         run_step(layers, dynamic=dyn)
     graph.replay()
-    graph_ms = time_per_step(graph.replay, side_steps, flush, stream)
+    graph_ms = time_per_step(graph.replay, side_steps, flush, stream, clean)
     del graph
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out in the graph replays")
     for _ in range(3):
         baseline_step(layers)
-    base_ms = time_per_step(lambda: baseline_step(layers), side_steps, flush, stream)
+    base_ms = time_per_step(lambda: baseline_step(layers), side_steps, flush, stream, clean)
     graph_ms = max_over_ranks(graph_ms, dev)
     base_ms = max_over_ranks(base_ms, dev)
     out = {
@@ -311,7 +321,8 @@ def gpu_arm(args, rank, world, dev):
                    "layers": [f"{L['spec'].M}x{L['spec'].K}x{L['spec'].N} r={L['spec'].r}"
                               + (" swiglu" if L["spec"].swiglu else "") + (" bias" if L["spec"].bias else "")
                               for L in layers],
-                   "l2": "flushed between timed steps (256 MB write, outside the events)",
+                   "l2": "flushed between timed steps (256 MB write" + (", then a 256 MB read" if args.l2_clean else "")
+                         + ", outside the events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "lora_rank": args.lora,
                    "activation_scale": "dynamic (amax pass every step)" if dyn else "static (calibrated once)"},
@@ -409,6 +420,7 @@ def fp8r_arm(args, dev):
             prev_out = Y
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if args.l2_clean else None
 
     def step(ev=None):
         for i, L in enumerate(layers):
@@ -432,7 +444,7 @@ def fp8r_arm(args, dev):
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         for s in range(K):
-            flush.zero_()
+            flush_l2(flush, clean)
             se[s][0].record(stream)
             step(kev[s])
             se[s][1].record(stream)
@@ -476,7 +488,7 @@ def fp8r_side(args):
     """fp8r_arm in a child process (its own CUDA context and a time limit), so that nothing in it can
     affect the main measurement; any failure comes back as {"error": ...}."""
     cmd = [sys.executable, os.path.abspath(__file__), "--fp8r-only", "--workload", args.workload,
-           "--steps", str(max(3, min(args.steps, 50))), "--warmup", "3"]
+           "--steps", str(max(3, min(args.steps, 50))), "--warmup", "3"] + (["--l2-clean"] if getattr(args, "l2_clean", False) else [])
     try:
         r = subprocess.run(cmd, capture_output=True, text=True, timeout=900, cwd=ROOT)
         lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
@@ -594,6 +606,8 @@ def main():
     ap.add_argument("--lora", type=int, default=0,
                     help="rank of a synthetic LoRA adapter concatenated onto each layer's branch")
     ap.add_argument("--no-fp8r", action="store_true", help="skip the row-wise FP8 side measurement")
+    ap.add_argument("--l2-clean", action="store_true",
+                    help="after each 256 MB write-flush also read 256 MB, so steps start with clean L2 lines")
     ap.add_argument("--fp8r-only", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
