@@ -360,3 +360,17 @@ def test_mlp_fused_argument_checks(L):
     if not torch.cuda.is_available():
         a, w, wn, an = _fake_mlp(L)
         assert _call_mlp(L, a, w, wn, an) == 3, L.svdq_last_error()  # well-formed: stops at the device
+
+
+def test_binding_refuses_cpu_tensors():
+    """No CPU fallback in the binding either: host tensors are refused before any library call."""
+    import torch
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+    R, inv = torch.zeros(128, 256), torch.ones(256)
+    L1, L2 = torch.zeros(256, 16, dtype=torch.bfloat16), torch.zeros(16, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        svdq.PackedWeight(R, L1, L2, inv)
+    with pytest.raises(ValueError, match="CUDA"):
+        svdq.Fp8rWeight(R, L1, L2, inv)
+    with pytest.raises(ValueError, match="CUDA"):
+        svdq.PackedWeight(R.double(), L1, L2, inv)          # and the wrong dtype
