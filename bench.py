@@ -9,7 +9,8 @@ write) between timed steps, outside the timed events. Timing: CUDA events on the
                   [--dynamic-scale] [--lora R] [--no-fp8r] [--no-cpu-baseline] [--l2-clean]
 
 On one GPU the line also carries the row-wise FP8 variant of the same workload, measured in a
-child process under the same protocol (``fp8r_variant``).
+child process under the same protocol (``fp8r_variant``), and for the MLP workloads the chain with
+the down layer's kernel 1 fused into the gate/up GEMM's epilogue (``mlp_fused``).
 
 N > 1 runs under torchrun as independent replicas (the layer has no exchange step), weak scaling.
 Prints one JSON line on rank 0.
@@ -485,9 +486,77 @@ def fp8r_arm(args, dev):
 
 
 def fp8r_side(args):
-    """fp8r_arm in a child process (its own CUDA context and a time limit), so that nothing in it can
-    affect the main measurement; any failure comes back as {"error": ...}."""
-    cmd = [sys.executable, os.path.abspath(__file__), "--fp8r-only", "--workload", args.workload,
+    """fp8r_arm in a child process (see child_side)."""
+    return child_side(args, "--fp8r-only")
+
+
+# ------------------------------------------------------------------ MLP chain with kernel 1 fused
+def mlp_fused_arm(args, dev):
+    """The MLP workload with the down layer's kernel 1 fused into the gate/up GEMM's SwiGLU epilogue:
+    per step kernel 1 of the gate/up layer, the fused GEMM (+ its small finalize pass) and the down
+    GEMM; h does not cross HBM. Same timing protocol. Also the relative difference of the down
+    layer's output from the unfused chain's, on the same inputs and scales."""
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+
+    wl = synth.WORKLOADS[args.workload]
+    up, dn = build_layers(wl, dev)                # the unfused chain: h -> Y of the first layer
+    scratch = torch.empty(svdq._lib.lib().svdq_mlp_scratch_bytes(up["spec"].M, dn["spec"].r), dtype=torch.uint8,
+                          device=dev)
+    act_dn = svdq.QuantizedAct(dn["spec"].M, dn["spec"].K, dn["spec"].r, dev)
+    Y = torch.empty_like(dn["Y"])
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if args.l2_clean else None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        svdq.quantize_act(up["X"], up["w"], up["g_x"], up["act"])
+        if ev is not None:
+            ev[1].record(stream)
+        svdq.gemm_swiglu_quant(up["act"], up["w"], up["bias"], dn["w"], dn["g_x"], act_dn, scratch)
+        if ev is not None:
+            ev[2].record(stream)
+        svdq.gemm(act_dn, dn["w"], dn["bias"], out=Y)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out during the fused warm-up")
+    # the unfused chain on the same inputs and scales, for the difference figure
+    run_step([up, dn])
+    torch.cuda.synchronize(dev)
+    ref = dn["Y"].float()
+    diff = float((Y.float() - ref).norm() / ref.norm())
+    K = args.steps
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        for s in range(K):
+            flush_l2(flush, clean)
+            step(ev[s])
+        torch.cuda.synchronize(dev)
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out in the fused timed region")
+    ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
+    part = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(3)]
+    flops = layer_flops(up["spec"])[0] + layer_flops(dn["spec"])[0]
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+            "steps": K, "warmup": args.warmup,
+            "kernels_us": {"quantize_act_up": round(part[0] * 1e3, 2), "gemm_swiglu_quant": round(part[1] * 1e3, 2),
+                           "gemm_down": round(part[2] * 1e3, 2)},
+            "rel_diff_vs_unfused_chain": round(diff, 7), "gpu_launches": 4 * K, "clocks": clk.summary(),
+            "what": "gate/up GEMM with the down layer's kernel 1 fused into its SwiGLU epilogue, then the down "
+                    "GEMM; run in a separate process"}
+
+
+def child_side(args, flag):
+    """An arm of this script in a child process (its own CUDA context and a time limit), so that
+    nothing in it can affect the main measurement; any failure comes back as {"error": ...}."""
+    cmd = [sys.executable, os.path.abspath(__file__), flag, "--workload", args.workload,
            "--steps", str(max(3, min(args.steps, 50))), "--warmup", "3"] + (["--l2-clean"] if getattr(args, "l2_clean", False) else [])
     try:
         r = subprocess.run(cmd, capture_output=True, text=True, timeout=900, cwd=ROOT)
@@ -609,6 +678,9 @@ def main():
     ap.add_argument("--l2-clean", action="store_true",
                     help="after each 256 MB write-flush also read 256 MB, so steps start with clean L2 lines")
     ap.add_argument("--fp8r-only", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--mlp-fused-only", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--no-mlp-fused", action="store_true",
+                    help="skip the fused-chain side measurement of the MLP workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -627,6 +699,9 @@ def main():
     if args.fp8r_only:
         print(json.dumps(fp8r_arm(args, dev)), flush=True)
         return
+    if args.mlp_fused_only:
+        print(json.dumps(mlp_fused_arm(args, dev)), flush=True)
+        return
     if world > 1:
         from datetime import timedelta
         torch.distributed.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
@@ -635,6 +710,8 @@ def main():
         if rank == 0:
             if world == 1 and not args.no_fp8r:
                 out["fp8r_variant"] = fp8r_side(args)
+            if world == 1 and args.workload.startswith("mlp") and not args.no_mlp_fused:
+                out["mlp_fused"] = child_side(args, "--mlp-fused-only")
             if world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
             print(json.dumps(out), flush=True)
