@@ -1,0 +1,166 @@
+"""A discrete-event model of the barrier protocol of the NVFP4 CTA-pair GEMM (svdq_gemm_kernel in
+csrc/svdq_gemm.cuh), checked on the host like test_fused_protocol_model.py: producer, MMA issuer,
+the four scale-factor writer warps and the eight epilogue warps of both CTAs replay their barrier
+traffic in the kernel's order, with copies and MMA completions landing late and in random order.
+Both accumulator modes are covered: one 256- or 192-column buffer (5-stage ring), and two
+128-column buffers used alternately (6-stage ring), the mode whose multi-tile runs the full-size
+workloads do not reach. Checked: no deadlock, no stray arrival, waits on exactly their completion,
+no resource used before its previous user is done; removing any one wait must make it fail."""
+import random
+
+import pytest
+
+SF_BUFS = 4
+WAITS = ["producer.empty", "issuer.acce", "issuer.sf_full", "sf.full", "sf.release", "epi.accf"]
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.completed = name, count, count, 0
+
+    def arrive(self, n=1):
+        self.pending -= n
+        assert self.pending >= 0, f"{self.name}: more arrivals than its count in one phase"
+        if self.pending == 0:
+            self.completed += 1
+            self.pending = self.count
+
+
+def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
+    rng = random.Random(seed)
+    slots = (r + 31) // 32 + k_iters
+    B = {}
+
+    def bar(name, count):
+        B[name] = Barrier(name, count)
+
+    for c in (0, 1):
+        for s in range(stages):
+            bar(f"full{c}.{s}", 1)
+            bar(f"empty{c}.{s}", 1)
+        for a in range(acc_bufs):
+            bar(f"accf{c}.{a}", 1)
+    for a in range(acc_bufs):
+        bar(f"acce{a}", 16)
+    for b in range(SF_BUFS):
+        bar(f"sf_full{b}", 8)
+    done = lambda name: B[name].completed  # noqa: E731
+    in_flight = []
+
+    def wait(tag, name, index):
+        if tag in skip:
+            return
+        while (B[name].completed & 1) == (index & 1):
+            yield name
+        assert B[name].completed == index + 1, \
+            f"{name}: wait for completion #{index} passed at completed = {B[name].completed}"
+
+    def producer(c):
+        uses = [0] * stages
+        stage = 0
+        for _ in range(n_tiles * slots):
+            yield from wait("producer.empty", f"empty{c}.{stage}", uses[stage] - 1)
+            assert done(f"empty{c}.{stage}") >= uses[stage], "ring stage refilled while its MMAs read it"
+            uses[stage] += 1
+            in_flight.append(f"full{c}.{stage}")
+            stage = (stage + 1) % stages
+
+    def issuer():
+        stage, sfb, g = 0, 0, 0
+        sf_uses = [0] * SF_BUFS
+        for t in range(n_tiles):
+            a, use = t % acc_bufs, t // acc_bufs
+            yield from wait("issuer.acce", f"acce{a}", use - 1)
+            assert done(f"acce{a}") >= use, "accumulator overwritten before its epilogue read it"
+            for _ in range(slots):
+                yield from wait("issuer.sf_full", f"sf_full{sfb}", sf_uses[sfb])
+                sf_uses[sfb] += 1
+                for c in (0, 1):
+                    assert done(f"full{c}.{stage}") >= g // stages + 1, "MMA before a CTA's copy landed"
+                for c in (0, 1):
+                    in_flight.append(f"empty{c}.{stage}")
+                stage = (stage + 1) % stages
+                sfb = (sfb + 1) % SF_BUFS
+                g += 1
+            for c in (0, 1):
+                in_flight.append(f"accf{c}.{a}")
+
+    def sf_writers(c):
+        full_uses = [0] * stages
+        released = [0] * stages
+        stage, sfb, n = 0, 0, 0
+        for _ in range(n_tiles * slots):
+            yield from wait("sf.full", f"full{c}.{stage}", full_uses[stage])
+            full_uses[stage] += 1
+            if n >= SF_BUFS:
+                ps = (stage - SF_BUFS) % stages
+                yield from wait("sf.release", f"empty{c}.{ps}", released[ps])
+                released[ps] += 1
+            B[f"sf_full{sfb}"].arrive(4)
+            n += 1
+            stage = (stage + 1) % stages
+            sfb = (sfb + 1) % SF_BUFS
+
+    def epilogue(c):
+        for t in range(n_tiles):
+            a, use = t % acc_bufs, t // acc_bufs
+            yield from wait("epi.accf", f"accf{c}.{a}", use)
+            assert done(f"accf{c}.{a}") >= use + 1, "accumulator read before its MMAs completed"
+            B[f"acce{a}"].arrive()
+
+    live = {"issuer": issuer()}
+    for c in (0, 1):
+        live[f"producer{c}"] = producer(c)
+        live[f"sf{c}"] = sf_writers(c)
+        for w in range(8):
+            live[f"epi{c}.{w}"] = epilogue(c)
+
+    for _ in range(1_000_000):
+        if not live:
+            break
+        waiting = {}
+        for k in rng.sample(sorted(live), len(live)):
+            try:
+                waiting[k] = next(live[k])
+            except StopIteration:
+                del live[k]
+        if live and not in_flight and all(waiting.get(k) is not None for k in live):
+            still = {}
+            for k in list(live):
+                try:
+                    still[k] = next(live[k])
+                except StopIteration:
+                    del live[k]
+            if live and not in_flight and all(v is not None for v in still.values()):
+                raise AssertionError(f"deadlock: {still}")
+        rng.shuffle(in_flight)
+        for _ in range(rng.randint(0, len(in_flight))):
+            B[in_flight.pop()].arrive()
+    assert not live, "model did not finish"
+    while in_flight:
+        B[in_flight.pop()].arrive()
+    for name, b in B.items():
+        assert b.pending == b.count, f"{name}: {b.count - b.pending} stray arrivals at the end"
+    return True
+
+
+# (stages, accumulator buffers) of the kernel's instantiations: 256 and 192 -> (5, 1), 128 -> (6, 2)
+@pytest.mark.parametrize("stages,acc_bufs", [(5, 1), (6, 2)])
+@pytest.mark.parametrize("n_tiles", [1, 2, 3, 8])
+@pytest.mark.parametrize("r,k_iters", [(32, 1), (64, 2), (0, 3), (16, 12)])
+def test_nvfp4_protocol_model(stages, acc_bufs, n_tiles, r, k_iters):
+    for seed in range(5):
+        assert run_model(n_tiles, r, k_iters, stages, acc_bufs, seed)
+
+
+@pytest.mark.parametrize("skipped", WAITS)
+@pytest.mark.parametrize("stages,acc_bufs", [(5, 1), (6, 2)])
+def test_every_wait_is_needed(skipped, stages, acc_bufs):
+    for n_tiles in (3, 8):
+        for r, k_iters in ((32, 1), (0, 3), (16, 12)):
+            for seed in range(20):
+                try:
+                    run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip={skipped})
+                except AssertionError:
+                    return
+    pytest.fail(f"removing the wait {skipped} went unnoticed")
