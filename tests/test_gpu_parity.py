@@ -223,3 +223,14 @@ def test_multi_tile_per_pair(cuda_device, M, K, N, r, bias, swiglu):
     c.check_weight_codes()
     c.check_act_codes()
     c.check_outputs()
+
+
+@pytest.mark.parametrize("M", [127, 128, 129, 255, 256])
+def test_row_block_boundaries(cuda_device, M):
+    """M on either side of a 128-row block and of a 256-row pair: a partial block, an exact pair, a
+    pair whose odd CTA has no rows, and one block plus a row."""
+    X, W, b = _rand_layer(M, 256, 256, 16, seed=1000 + M, bias=True)
+    c = Case(X, W, b, 16, False, cuda_device)
+    c.check_scales()
+    c.check_act_codes()
+    c.check_outputs()
