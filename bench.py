@@ -559,7 +559,7 @@ def child_side(args, flag):
     cmd = [sys.executable, os.path.abspath(__file__), flag, "--workload", args.workload,
            "--steps", str(max(3, min(args.steps, 50))), "--warmup", "3"] + (["--l2-clean"] if getattr(args, "l2_clean", False) else [])
     try:
-        r = subprocess.run(cmd, capture_output=True, text=True, timeout=900, cwd=ROOT)
+        r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
         lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
         if r.returncode != 0 or not lines:
             return {"error": f"exit {r.returncode}: {(r.stderr or r.stdout)[-600:]}"}
