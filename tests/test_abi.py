@@ -1,6 +1,7 @@
 """The C-ABI library builds, loads without a GPU, exports every entry point include/svdq.h declares,
 and its host-side logic (size queries, layouts, argument checks) behaves; no compute call is made."""
 import ctypes
+import os
 
 import pytest
 
@@ -374,3 +375,63 @@ def test_binding_refuses_cpu_tensors():
         svdq.Fp8rWeight(R, L1, L2, inv)
     with pytest.raises(ValueError, match="CUDA"):
         svdq.PackedWeight(R.double(), L1, L2, inv)          # and the wrong dtype
+
+
+C_PROGRAM = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "svdq.h"
+int main(void) {
+  svdq_act act;
+  unsigned char* base = (unsigned char*)0 + ((size_t)1 << 40);
+  size_t nb = svdq_act_bytes(300, 512, 16);
+  svdq_status st = svdq_act_bind(300, 512, 16, base, nb, &act);
+  svdq_weight w;
+  float* p = (float*)((size_t)1 << 41);
+  svdq_status st2 = svdq_pack_weight(p, (const uint16_t*)p, (const uint16_t*)p, p, 512, 512, 16, 0, p,
+                                     (size_t)1 << 30, &w, NULL);
+  printf("%d %zu %zu %zu %d %d %d %zu %zu %d %zu %zu %zu %zu %s\n", svdq_abi_version(),
+         svdq_weight_bytes(9216, 3072, 32), nb, svdq_fp8r_weight_bytes(9216, 3072, 32), (int)st, act.M_pad,
+         (int)(act.scales != NULL), svdq_mlp_scratch_bytes(4608, 32), sizeof(svdq_weight), (int)st2,
+         sizeof(svdq_act), sizeof(svdq_fp8r_weight), sizeof(svdq_fp8r_act),
+         offsetof(svdq_weight, tmap), svdq_status_str(st2));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(L, tmp_path):
+    """include/svdq.h compiles as C99 and a C program links against libsvdq.so and runs its
+    host-only calls; the answers agree with the ctypes binding, and a compute call without a GPU
+    fails with SVDQ_ERR_CUDA."""
+    import shutil
+    import subprocess
+    import torch
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.dirname(_lib.HEADER),
+                        str(src), "-L", libdir, "-lsvdq", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    f = out.stdout.split()
+    assert int(f[0]) == L.svdq_abi_version()
+    assert int(f[1]) == L.svdq_weight_bytes(9216, 3072, 32)
+    assert int(f[2]) == L.svdq_act_bytes(300, 512, 16)
+    assert int(f[3]) == L.svdq_fp8r_weight_bytes(9216, 3072, 32)
+    assert int(f[4]) == 0 and int(f[5]) == 384 and int(f[6]) == 1
+    assert int(f[7]) == L.svdq_mlp_scratch_bytes(4608, 32)
+    # the ctypes layouts match C's
+    assert int(f[8]) == ctypes.sizeof(_lib.SvdqWeight)
+    assert int(f[10]) == ctypes.sizeof(_lib.SvdqAct)
+    assert int(f[11]) == ctypes.sizeof(_lib.SvdqFp8rWeight)
+    assert int(f[12]) == ctypes.sizeof(_lib.SvdqFp8rAct)
+    assert int(f[13]) == _lib.SvdqWeight.tmap.offset
+    if not torch.cuda.is_available():
+        assert int(f[9]) == 3                                    # SVDQ_ERR_CUDA: no fallback
