@@ -20,6 +20,9 @@
  *                         256-row tile (TMA-fed shared-memory rings, TMEM accumulators) whose
  *                         epilogue adds the up-projection U L2 (bf16 MMAs into the same
  *                         accumulator), bias and SwiGLU before one store.
+ * Further down: the row-wise FP8 (W8A8) variant of the same layer (svdq_fp8r_*), and the MLP
+ * chain's call that fuses the down layer's activation quantization into the gate/up GEMM's
+ * SwiGLU epilogue (svdq_gemm_swiglu_quant).
  *
  * Conventions for every entry point:
  *   - Pointers named as device memory must be device pointers on the current device; the library
