@@ -73,6 +73,7 @@ def _declare(lib):
         "svdq_pack_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,
                                      c_size_t, W, c_void_p]),
         "svdq_act_bind": (c_int, [c_int, c_int, c_int, c_void_p, c_size_t, A]),
+        "svdq_weight_bind": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p, c_size_t, W]),
         "svdq_calibrate_act": (c_int, [c_void_p, c_int, W, c_void_p, c_void_p]),
         "svdq_quantize_act": (c_int, [c_void_p, W, c_void_p, A, c_void_p]),
         "svdq_gemm": (c_int, [A, W, c_void_p, c_int, c_void_p, c_int, c_void_p]),
@@ -159,6 +160,29 @@ class PackedWeight:
     @property
     def n_tile(self) -> int:
         return self.desc.n_tile
+
+    def state_dict(self) -> dict:
+        """The packed blob (on the host) and the shape fields needed to re-bind it: a checkpoint of
+        the quantized weight that does not need R, the branch factors or the pack kernels again."""
+        return {"abi": lib().svdq_abi_version(), "N": self.N, "K": self.K, "r": self.r, "swiglu": self.swiglu,
+                "n_tile": self.n_tile, "blob": self.buf.cpu()}
+
+    @classmethod
+    def from_state(cls, state: dict, device) -> "PackedWeight":
+        """A packed weight from state_dict() output, copied to `device` and re-bound (its TMA
+        descriptors re-encoded for the new address)."""
+        if state["abi"] != lib().svdq_abi_version():
+            raise ValueError(f"checkpoint ABI {state['abi']} != library ABI {lib().svdq_abi_version()}")
+        self = cls.__new__(cls)
+        self.device = torch.device(device)
+        self.buf = state["blob"].to(self.device)
+        self.desc = SvdqWeight()
+        self.N, self.K, self.r, self.swiglu = state["N"], state["K"], state["r"], state["swiglu"]
+        with torch.cuda.device(self.device):
+            _check("svdq_weight_bind", lib().svdq_weight_bind(self.N, self.K, self.r, 1 if self.swiglu else 0,
+                                                              state["n_tile"], _ptr(self.buf), self.buf.numel(),
+                                                              byref(self.desc)))
+        return self
 
     def g_w(self) -> torch.Tensor:
         off = self.desc.g_w - self.buf.data_ptr()

@@ -377,6 +377,50 @@ svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const ui
   return SVDQ_OK;
 }
 
+svdq_status svdq_weight_bind(int N, int K, int r, int swiglu, int n_tile, void* blob, size_t blob_bytes,
+                             svdq_weight* out) {
+  if (out == nullptr || blob == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (N <= 0 || K <= 0 || K % 256 != 0 || K > (1 << 20) || N > (1 << 20) || !valid_r(r) ||
+      (n_tile != 256 && n_tile != 192 && n_tile != 128) || N % n_tile != 0)
+    return fail(SVDQ_ERR_UNSUPPORTED, "weight shape N=%d K=%d r=%d n_tile=%d unsupported", N, K, r, n_tile);
+  if (reinterpret_cast<uintptr_t>(blob) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "blob not 256-byte aligned");
+  const WeightLayout l = weight_layout(N, K, r, n_tile);
+  if (blob_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "weight blob %zu bytes < %zu", blob_bytes, l.total);
+  int dev, sms;
+  if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
+  uint8_t* b = static_cast<uint8_t*>(blob);
+  svdq_weight w{};
+  w.N = N;
+  w.K = K;
+  w.r = r;
+  w.swiglu_interleaved = swiglu ? 1 : 0;
+  w.n_tile = n_tile;
+  w.codes = b + l.codes;
+  w.scales = b + l.scales;
+  w.g_w = reinterpret_cast<float*>(b + l.gw);
+  w.inv_lambda = reinterpret_cast<float*>(b + l.inv_lambda);
+  w.L1s_t = b + l.l1t;
+  w.L2_t = b + l.l2t;
+  // the TMA descriptors hold absolute addresses: encode them for this copy of the blob, exactly as
+  // svdq_pack_weight does
+  CUtensorMap tmB, tmL2;
+  std::memset(&tmL2, 0, sizeof(tmL2));
+  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K / 2, N, K / 2, 128, n_tile / 2,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, N, static_cast<uint64_t>(r) * 2,
+                                  r < 32 ? r : 32, n_tile / 2, lr_swizzle(r));
+        s != SVDQ_OK)
+      return s;
+  }
+  std::memcpy(&w.tmap[0][0], &tmB, sizeof(CUtensorMap));
+  std::memcpy(&w.tmap[1][0], &tmL2, sizeof(CUtensorMap));
+  *out = w;
+  return SVDQ_OK;
+}
+
 svdq_status svdq_calibrate_act(const uint16_t* X, int M, const svdq_weight* w, float* g_x_out, svdq_stream_t stream) {
   if (X == nullptr || w == nullptr || g_x_out == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
   if (svdq_status s = check_weight(w); s != SVDQ_OK) return s;

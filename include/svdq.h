@@ -128,6 +128,15 @@ SVDQ_API svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr,
                              const float* inv_lambda, int N, int K, int r, int swiglu,
                              void* dst, size_t dst_bytes, svdq_weight* out, svdq_stream_t stream);
 
+/* Checkpoints: re-bind a packed weight blob without re-packing, e.g. one written by
+ * svdq_pack_weight, saved, and copied back to device memory. N, K, r, swiglu and n_tile are the
+ * values of the descriptor the blob was packed with (n_tile is not re-derived: an SVDQ_N_TILE
+ * override at pack time stays valid). The blob is 256-byte aligned and at least the packed size
+ * for those values. Fills `out` with pointers into `blob` and re-encodes its TMA descriptors for
+ * this address. */
+SVDQ_API svdq_status svdq_weight_bind(int N, int K, int r, int swiglu, int n_tile, void* blob, size_t blob_bytes,
+                             svdq_weight* out);
+
 /* Host-only: lay an svdq_act out over `dst` (device, >= svdq_act_bytes(M,K,r), 256-aligned). */
 SVDQ_API svdq_status svdq_act_bind(int M, int K, int r, void* dst, size_t dst_bytes, svdq_act* out);
 

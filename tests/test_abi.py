@@ -435,3 +435,20 @@ def test_header_is_plain_c_and_links(L, tmp_path):
     assert int(f[13]) == _lib.SvdqWeight.tmap.offset
     if not torch.cuda.is_available():
         assert int(f[9]) == 3                                    # SVDQ_ERR_CUDA: no fallback
+
+
+def test_weight_bind_checks(L):
+    """svdq_weight_bind (checkpoint reload): host checks first; a well-formed call stops at the
+    device query without a GPU."""
+    import torch
+    w = _lib.SvdqWeight()
+    p = ctypes.c_void_p(1 << 40)
+    need = _weight_bytes_for_tile(768, 512, 32, 128)
+    assert L.svdq_weight_bind(768, 512, 32, 0, 128, None, need, ctypes.byref(w)) == 1        # null blob
+    assert L.svdq_weight_bind(768, 512, 32, 0, 96, p, need, ctypes.byref(w)) == 2            # bad n_tile
+    assert L.svdq_weight_bind(640, 512, 32, 0, 256, p, need, ctypes.byref(w)) == 2           # 640 % 256
+    assert L.svdq_weight_bind(768, 500, 32, 0, 128, p, need, ctypes.byref(w)) == 2           # K % 256
+    assert L.svdq_weight_bind(768, 512, 32, 0, 128, ctypes.c_void_p((1 << 40) + 16), need, ctypes.byref(w)) == 2
+    assert L.svdq_weight_bind(768, 512, 32, 0, 128, p, need - 1, ctypes.byref(w)) == 1       # blob too small
+    if not torch.cuda.is_available():
+        assert L.svdq_weight_bind(768, 512, 32, 0, 128, p, need, ctypes.byref(w)) == 3

@@ -234,3 +234,18 @@ def test_row_block_boundaries(cuda_device, M):
     c.check_scales()
     c.check_act_codes()
     c.check_outputs()
+
+
+def test_packed_weight_checkpoint_round_trip(cuda_device):
+    """A packed weight saved to the host (state_dict) and re-bound at another device address
+    (from_state, svdq_weight_bind) gives the GEMM bit-identical outputs; SwiGLU packing included."""
+    for swiglu in (False, True):
+        X, W, b = _rand_layer(300, 512, 768, 32, seed=77 + swiglu, bias=True)
+        c = Case(X, W, b, 32, swiglu, cuda_device)
+        y0 = c.run_gemm(torch.float32)
+        restored = svdq.PackedWeight.from_state(c.w.state_dict(), cuda_device)
+        assert restored.buf.data_ptr() != c.w.buf.data_ptr()
+        y1 = svdq.gemm(c.act, restored, c.bias_d, out_dtype=torch.float32)
+        torch.cuda.synchronize(cuda_device)
+        assert svdq.device_status() == 0
+        assert torch.equal(y0, y1)
