@@ -70,6 +70,7 @@ def _declare(lib):
         "svdq_gemm_swiglu_quant": (c_int, [A, W, c_void_p, W, c_void_p, A, c_void_p, c_size_t, c_void_p, c_void_p]),
         "svdq_weight_bytes": (c_size_t, [c_int, c_int, c_int]),
         "svdq_act_bytes": (c_size_t, [c_int, c_int, c_int]),
+        "svdq_weight_bytes_tiled": (c_size_t, [c_int, c_int, c_int, c_int]),
         "svdq_pack_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,
                                      c_size_t, W, c_void_p]),
         "svdq_act_bind": (c_int, [c_int, c_int, c_int, c_void_p, c_size_t, A]),
@@ -173,9 +174,17 @@ class PackedWeight:
         descriptors re-encoded for the new address)."""
         if state["abi"] != lib().svdq_abi_version():
             raise ValueError(f"checkpoint ABI {state['abi']} != library ABI {lib().svdq_abi_version()}")
+        blob = state["blob"]
+        if not isinstance(blob, torch.Tensor) or blob.dtype != torch.uint8 or blob.dim() != 1 \
+                or not blob.is_contiguous():
+            raise ValueError("checkpoint blob: expected a contiguous one-dimensional uint8 tensor")
+        need = lib().svdq_weight_bytes_tiled(state["N"], state["K"], state["r"], state["n_tile"])
+        if need == 0 or blob.numel() != need:
+            raise ValueError(f"checkpoint blob holds {blob.numel()} bytes; a weight packed with N={state['N']} "
+                             f"K={state['K']} r={state['r']} n_tile={state['n_tile']} holds {need}")
         self = cls.__new__(cls)
         self.device = torch.device(device)
-        self.buf = state["blob"].to(self.device)
+        self.buf = blob.to(self.device)
         self.desc = SvdqWeight()
         self.N, self.K, self.r, self.swiglu = state["N"], state["K"], state["r"], state["swiglu"]
         with torch.cuda.device(self.device):

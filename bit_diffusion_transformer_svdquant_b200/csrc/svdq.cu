@@ -237,6 +237,43 @@ svdq_status check_act(const svdq_act* a) {
   return SVDQ_OK;
 }
 
+// Descriptor of a packed weight blob at `b`: the pointers of weight_layout(N, K, r, n_tile) and
+// the TMA descriptors of its codes and L2^T, which hold absolute addresses and so are encoded for
+// this copy of the blob. svdq_pack_weight and svdq_weight_bind both fill descriptors here.
+svdq_status fill_weight_desc(uint8_t* b, int N, int K, int r, int swiglu, int n_tile, svdq_weight* out) {
+  const WeightLayout l = weight_layout(N, K, r, n_tile);
+  svdq_weight w{};
+  w.N = N;
+  w.K = K;
+  w.r = r;
+  w.swiglu_interleaved = swiglu ? 1 : 0;
+  w.n_tile = n_tile;
+  w.codes = b + l.codes;
+  w.scales = b + l.scales;
+  w.g_w = reinterpret_cast<float*>(b + l.gw);
+  w.inv_lambda = reinterpret_cast<float*>(b + l.inv_lambda);
+  w.L1s_t = b + l.l1t;
+  w.L2_t = b + l.l2t;
+  static_assert(sizeof(w.tmap) >= 2 * sizeof(CUtensorMap), "tmap storage");
+  CUtensorMap tmB, tmL2;
+  std::memset(&tmL2, 0, sizeof(tmL2));
+  // each CTA of a GEMM pair stages half of a tile's n_tile rows
+  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K / 2, N, K / 2, 128, n_tile / 2,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+      s != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, N, static_cast<uint64_t>(r) * 2,
+                                  r < 32 ? r : 32, n_tile / 2, lr_swizzle(r));
+        s != SVDQ_OK)
+      return s;
+  }
+  std::memcpy(&w.tmap[0][0], &tmB, sizeof(CUtensorMap));
+  std::memcpy(&w.tmap[1][0], &tmL2, sizeof(CUtensorMap));
+  *out = w;
+  return SVDQ_OK;
+}
+
 int grid_for(size_t work_items, int per_block, int sm_count) {
   size_t blocks = (work_items + per_block - 1) / per_block;
   size_t cap = static_cast<size_t>(sm_count) * 16;
@@ -273,6 +310,13 @@ const char* svdq_last_error(void) { return g_last_error.c_str(); }
 size_t svdq_weight_bytes(int N, int K, int r) {
   if (!shape_ok(N, K, r)) return 0;
   return weight_layout(N, K, r, choose_n_tile(N)).total;
+}
+
+size_t svdq_weight_bytes_tiled(int N, int K, int r, int n_tile) {
+  if (N <= 0 || K <= 0 || K % 256 != 0 || K > (1 << 20) || N > (1 << 20) || !valid_r(r) ||
+      (n_tile != 256 && n_tile != 192 && n_tile != 128) || N % n_tile != 0)
+    return 0;
+  return weight_layout(N, K, r, n_tile).total;
 }
 
 size_t svdq_act_bytes(int M, int K, int r) {
@@ -325,17 +369,7 @@ svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const ui
   uint8_t* b = static_cast<uint8_t*>(dst);
 
   svdq_weight w{};
-  w.N = N;
-  w.K = K;
-  w.r = r;
-  w.swiglu_interleaved = swiglu ? 1 : 0;
-  w.n_tile = n_tile;
-  w.codes = b + l.codes;
-  w.scales = b + l.scales;
-  w.g_w = reinterpret_cast<float*>(b + l.gw);
-  w.inv_lambda = reinterpret_cast<float*>(b + l.inv_lambda);
-  w.L1s_t = b + l.l1t;
-  w.L2_t = b + l.l2t;
+  if (svdq_status s = fill_weight_desc(b, N, K, r, swiglu, n_tile, &w); s != SVDQ_OK) return s;
 
   SVDQ_CUDA(cudaMemsetAsync(b + l.scales, 0, l.gw - l.scales + 4, st));  // pad rows of the scale layout, amax
   SVDQ_CUDA(cudaMemcpyAsync(w.inv_lambda, inv_lambda, static_cast<size_t>(K) * 4, cudaMemcpyDeviceToDevice, st));
@@ -357,22 +391,6 @@ svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const ui
         static_cast<__nv_bfloat16*>(w.L2_t));
     if (svdq_status s = check_launch("pack_l2_kernel"); s != SVDQ_OK) return s;
   }
-  static_assert(sizeof(w.tmap) >= 2 * sizeof(CUtensorMap), "tmap storage");
-  CUtensorMap tmB, tmL2;
-  std::memset(&tmL2, 0, sizeof(tmL2));
-  // each CTA of a GEMM pair stages half of a tile's n_tile rows
-  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K / 2, N, K / 2, 128, n_tile / 2,
-                                CU_TENSOR_MAP_SWIZZLE_128B);
-      s != SVDQ_OK)
-    return s;
-  if (r > 0) {
-    if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, N, static_cast<uint64_t>(r) * 2,
-                                  r < 32 ? r : 32, n_tile / 2, lr_swizzle(r));
-        s != SVDQ_OK)
-      return s;
-  }
-  std::memcpy(&w.tmap[0][0], &tmB, sizeof(CUtensorMap));
-  std::memcpy(&w.tmap[1][0], &tmL2, sizeof(CUtensorMap));
   *out = w;
   return SVDQ_OK;
 }
@@ -388,37 +406,8 @@ svdq_status svdq_weight_bind(int N, int K, int r, int swiglu, int n_tile, void* 
   if (blob_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "weight blob %zu bytes < %zu", blob_bytes, l.total);
   int dev, sms;
   if (svdq_status s = device_ready(&dev, &sms); s != SVDQ_OK) return s;
-  uint8_t* b = static_cast<uint8_t*>(blob);
-  svdq_weight w{};
-  w.N = N;
-  w.K = K;
-  w.r = r;
-  w.swiglu_interleaved = swiglu ? 1 : 0;
-  w.n_tile = n_tile;
-  w.codes = b + l.codes;
-  w.scales = b + l.scales;
-  w.g_w = reinterpret_cast<float*>(b + l.gw);
-  w.inv_lambda = reinterpret_cast<float*>(b + l.inv_lambda);
-  w.L1s_t = b + l.l1t;
-  w.L2_t = b + l.l2t;
-  // the TMA descriptors hold absolute addresses: encode them for this copy of the blob, exactly as
-  // svdq_pack_weight does
-  CUtensorMap tmB, tmL2;
-  std::memset(&tmL2, 0, sizeof(tmL2));
-  if (svdq_status s = make_tmap(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, K / 2, N, K / 2, 128, n_tile / 2,
-                                CU_TENSOR_MAP_SWIZZLE_128B);
-      s != SVDQ_OK)
-    return s;
-  if (r > 0) {
-    if (svdq_status s = make_tmap(&tmL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.L2_t, r, N, static_cast<uint64_t>(r) * 2,
-                                  r < 32 ? r : 32, n_tile / 2, lr_swizzle(r));
-        s != SVDQ_OK)
-      return s;
-  }
-  std::memcpy(&w.tmap[0][0], &tmB, sizeof(CUtensorMap));
-  std::memcpy(&w.tmap[1][0], &tmL2, sizeof(CUtensorMap));
-  *out = w;
-  return SVDQ_OK;
+  // the TMA descriptors hold absolute addresses: they are encoded for this copy of the blob
+  return fill_weight_desc(static_cast<uint8_t*>(blob), N, K, r, swiglu, n_tile, out);
 }
 
 svdq_status svdq_calibrate_act(const uint16_t* X, int M, const svdq_weight* w, float* g_x_out, svdq_stream_t stream) {

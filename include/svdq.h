@@ -111,6 +111,10 @@ typedef struct svdq_act {
 /* Bytes of device memory a packed weight / a quantized activation needs (0 on bad shapes). */
 SVDQ_API size_t svdq_weight_bytes(int N, int K, int r);
 SVDQ_API size_t svdq_act_bytes(int M, int K, int r);
+/* Bytes of a packed weight blob for an explicit GEMM tile width n_tile (256, 192 or 128; the
+ * value a descriptor's n_tile field holds), e.g. to check a checkpoint's blob before re-binding it
+ * with svdq_weight_bind. 0 on bad shapes or a tile width that does not divide N. */
+SVDQ_API size_t svdq_weight_bytes_tiled(int N, int K, int r, int n_tile);
 
 /* Offline pack of one layer's weight (not on the per-step path).
  *   R_nk        device fp32 [N][K]  residual R = W_hat - diag(lambda) L1s L2 (nn.Linear layout)

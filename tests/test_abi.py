@@ -452,3 +452,42 @@ def test_weight_bind_checks(L):
     assert L.svdq_weight_bind(768, 512, 32, 0, 128, p, need - 1, ctypes.byref(w)) == 1       # blob too small
     if not torch.cuda.is_available():
         assert L.svdq_weight_bind(768, 512, 32, 0, 128, p, need, ctypes.byref(w)) == 3
+
+
+@pytest.mark.parametrize("N,K,r,tile", [(768, 512, 32, 128), (768, 512, 32, 192), (768, 512, 32, 256),
+                                        (9216, 3072, 32, 256), (384, 256, 0, 192), (640, 1024, 64, 128)])
+def test_weight_bytes_tiled(L, N, K, r, tile):
+    """The size query with an explicit tile width gives the layout of that width."""
+    assert L.svdq_weight_bytes_tiled(N, K, r, tile) == _weight_bytes_for_tile(N, K, r, tile)
+
+
+def test_weight_bytes_tiled_rejects(L):
+    assert L.svdq_weight_bytes_tiled(768, 512, 32, 96) == 0       # not a tile width
+    assert L.svdq_weight_bytes_tiled(640, 512, 32, 256) == 0      # 256 does not divide 640
+    assert L.svdq_weight_bytes_tiled(768, 500, 32, 128) == 0      # K % 256
+    assert L.svdq_weight_bytes_tiled(768, 512, 24, 128) == 0      # rank
+
+
+def test_from_state_checks_the_blob(L):
+    """A checkpoint whose blob is not a contiguous 1-D uint8 tensor of exactly the packed size for its
+    N, K, r and n_tile is refused before anything is copied to a device."""
+    import torch
+    N, K, r, t = 768, 512, 32, 128
+    need = _weight_bytes_for_tile(N, K, r, t)
+    base = {"abi": L.svdq_abi_version(), "N": N, "K": K, "r": r, "swiglu": False, "n_tile": t}
+    bad = [
+        torch.zeros(need, dtype=torch.int8),                       # dtype changed on save / load
+        torch.zeros(need // 2, dtype=torch.int16),
+        torch.zeros(2, need // 2, dtype=torch.uint8),              # not one-dimensional
+        torch.zeros(2 * need, dtype=torch.uint8)[::2],             # not contiguous
+        torch.zeros(need + 256, dtype=torch.uint8),                # another layer's size
+        torch.zeros(need - 256, dtype=torch.uint8),
+    ]
+    for blob in bad:
+        with pytest.raises(ValueError, match="checkpoint blob"):
+            _lib.PackedWeight.from_state({**base, "blob": blob}, "cpu")
+    # fields of another layer (n_tile 192 over the 128-wide blob: 4 x 2 scale atoms per K step
+    # instead of 6 x 1) are refused too
+    assert _weight_bytes_for_tile(N, K, r, 192) != need
+    with pytest.raises(ValueError, match="checkpoint blob"):
+        _lib.PackedWeight.from_state({**base, "n_tile": 192, "blob": torch.zeros(need, dtype=torch.uint8)}, "cpu")

@@ -135,27 +135,36 @@ def test_full_size_workload(cuda_device, spec):
 
 def test_cuda_graph_replay(cuda_device):
     """Both kernels captured in a CUDA graph and replayed give the eager result bit for bit (the
-    library enqueues everything on the caller's stream and allocates nothing per call)."""
+    library enqueues everything on the caller's stream and allocates nothing per call), in bf16 and
+    fp32 output modes; the replayed activation codes and scales equal the oracle's, and the replayed
+    fp32 output is within 2e-3 of max|y_ref| of the oracle's layer."""
     X, W, b = _rand_layer(300, 768, 512, 32, seed=11, bias=True)
     c = Case(X, W, b, 32, False, cuda_device)
-    y_eager = c.run_gemm(torch.bfloat16).clone()
-    Y = torch.empty_like(y_eager)
-    side = torch.cuda.Stream(cuda_device)
-    side.wait_stream(torch.cuda.current_stream(cuda_device))
-    with torch.cuda.stream(side):
-        svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
-        svdq.gemm(c.act, c.w, c.bias_d, out=Y)
-    torch.cuda.current_stream(cuda_device).wait_stream(side)
-    Y.zero_()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
-        svdq.gemm(c.act, c.w, c.bias_d, out=Y)
-    Y.zero_()
-    g.replay()
-    torch.cuda.synchronize(cuda_device)
-    assert svdq.device_status() == 0
-    assert torch.equal(Y, y_eager)
+    for dt in (torch.bfloat16, torch.float32):
+        y_eager = c.run_gemm(dt).clone()
+        Y = torch.empty_like(y_eager)
+        side = torch.cuda.Stream(cuda_device)
+        side.wait_stream(torch.cuda.current_stream(cuda_device))
+        with torch.cuda.stream(side):
+            svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
+            svdq.gemm(c.act, c.w, c.bias_d, out=Y, out_dtype=dt)
+        torch.cuda.current_stream(cuda_device).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
+            svdq.gemm(c.act, c.w, c.bias_d, out=Y, out_dtype=dt)
+        Y.zero_()
+        c.act.buf.zero_()        # the replay must rewrite codes, scales, U and alpha itself
+        g.replay()
+        torch.cuda.synchronize(cuda_device)
+        assert svdq.device_status() == 0
+        assert torch.equal(Y, y_eager)
+        c.check_act_codes()
+        if dt == torch.float32:
+            y = Y.cpu().numpy().astype(np.float64)
+            ref = c.y_ref_full()
+            assert np.max(np.abs(y - ref)) <= 2e-3 * np.max(np.abs(ref))
+        del g
 
 
 def test_lora_on_the_branch(cuda_device):
@@ -236,16 +245,43 @@ def test_row_block_boundaries(cuda_device, M):
     c.check_outputs()
 
 
+_DESC_PTRS = ("codes", "scales", "g_w", "inv_lambda", "L1s_t", "L2_t")
+
+
 def test_packed_weight_checkpoint_round_trip(cuda_device):
     """A packed weight saved to the host (state_dict) and re-bound at another device address
-    (from_state, svdq_weight_bind) gives the GEMM bit-identical outputs; SwiGLU packing included."""
+    (from_state, svdq_weight_bind) gives the GEMM bit-identical outputs; SwiGLU packing included.
+    The original blob is overwritten before the restored weight runs, so a bind that kept the old
+    TMA descriptors (or pointers) would read garbage and fail."""
     for swiglu in (False, True):
         X, W, b = _rand_layer(300, 512, 768, 32, seed=77 + swiglu, bias=True)
         c = Case(X, W, b, 32, swiglu, cuda_device)
         y0 = c.run_gemm(torch.float32)
         restored = svdq.PackedWeight.from_state(c.w.state_dict(), cuda_device)
         assert restored.buf.data_ptr() != c.w.buf.data_ptr()
+        lo, hi = restored.buf.data_ptr(), restored.buf.data_ptr() + restored.buf.numel()
+        for f in _DESC_PTRS:
+            assert lo <= getattr(restored.desc, f) < hi, f
+        g = torch.Generator(device=cuda_device).manual_seed(5)
+        c.w.buf.copy_(torch.randint(0, 256, c.w.buf.shape, generator=g, device=cuda_device, dtype=torch.int32)
+                      .to(torch.uint8))
         y1 = svdq.gemm(c.act, restored, c.bias_d, out_dtype=torch.float32)
         torch.cuda.synchronize(cuda_device)
         assert svdq.device_status() == 0
         assert torch.equal(y0, y1)
+
+
+def test_weight_bind_offsets_match_pack(cuda_device):
+    """A bind of an (uninitialised) blob puts every descriptor pointer at the offset a pack into a
+    buffer of the same shape produces, relative to each buffer's start."""
+    X, W, b = _rand_layer(256, 512, 768, 32, seed=79, bias=False)
+    c = Case(X, W, None, 32, False, cuda_device)
+    blob = torch.empty_like(c.w.buf)
+    lib = svdq._lib.lib()
+    d = svdq._lib.SvdqWeight()
+    import ctypes
+    assert lib.svdq_weight_bind(c.w.N, c.w.K, c.w.r, 0, c.w.n_tile, ctypes.c_void_p(blob.data_ptr()),
+                                blob.numel(), ctypes.byref(d)) == 0
+    for f in _DESC_PTRS:
+        assert getattr(d, f) - blob.data_ptr() == getattr(c.w.desc, f) - c.w.buf.data_ptr(), f
+    assert (d.N, d.K, d.r, d.n_tile, d.swiglu_interleaved) == (c.w.N, c.w.K, c.w.r, c.w.n_tile, 0)

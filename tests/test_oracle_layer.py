@@ -174,3 +174,32 @@ def test_lora_on_the_branch_is_additive():
     l0 = svdquant.add_lora(p0, A, B)
     np.testing.assert_allclose(svdquant.layer_forward(X, l0, g_x, wq0),
                                svdquant.layer_forward(X, p0, g_x, wq0) + (X @ A) @ B, rtol=1e-12, atol=1e-12)
+
+
+def test_activation_scale_on_a_hand_example():
+    """The static activation scale is taken over the SMOOTHED activations: g_x = fp32(max|x *
+    inv_lambda| / 2688). Hand example (4 tokens x 32 channels, bf16-exact values): channel 3 is an
+    outlier channel (raw values up to 100) with inv_lambda = 1/4, so its smoothed values peak at 25;
+    channel 21 holds the smoothed maximum, x = -40 with inv_lambda = 1. So the smoothed amax is 40,
+    the raw amax 100, and the block of 16 channels holding (token 2, channel 21) is the one whose
+    E4M3 scale is 448 (code 0x7E). A scale computed on the unsmoothed X (100 / 2688) or with lambda
+    in place of 1 / lambda (100 * 4 / 2688) gives another value, so either mistake fails here."""
+    X = np.zeros((4, 32))
+    X[:, 0] = [1.5, -2.0, 0.5, 3.0]
+    X[:, 3] = [100.0, -96.0, 64.0, 80.0]
+    X[:, 21] = [12.0, 8.0, -40.0, 30.0]
+    X[:, 30] = [-6.0, 7.0, 2.0, -3.5]
+    inv_lambda = np.ones(32)
+    inv_lambda[3] = 0.25
+    inv_lambda[30] = 0.5
+    g_expected = float(np.float32(40.0 / 2688.0))
+    g = svdquant.calibrate_activation_scale(X, inv_lambda)
+    assert g == g_expected
+    assert g != float(np.float32(100.0 / 2688.0))        # raw amax
+    assert g != float(np.float32(400.0 / 2688.0))        # lambda instead of 1 / lambda
+    q, s = svdquant.quantize_activations(X, inv_lambda, g)
+    assert s.shape == (4, 2)
+    assert s[2, 1] == 0x7E                                # block (token 2, channels 16..31)
+    assert (s[[0, 1, 3], 1] < 0x7E).all() and (s[:, 0] < 0x7E).all()
+    # the amax element itself encodes to -6 (sign bit | code 7)
+    assert q[2, 21] == 0x8 | 0x7
