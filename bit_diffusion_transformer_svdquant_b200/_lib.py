@@ -68,6 +68,7 @@ def _declare(lib):
         "svdq_fp8r_export_act": (c_int, [FA, c_void_p, c_void_p, c_void_p]),
         "svdq_mlp_scratch_bytes": (c_size_t, [c_int, c_int]),
         "svdq_gemm_swiglu_quant": (c_int, [A, W, c_void_p, W, c_void_p, A, c_void_p, c_size_t, c_void_p, c_void_p]),
+        "svdq_gemm_swiglu_quant_noscratch": (c_int, [A, W, c_void_p, W, c_void_p, A, c_void_p, c_void_p]),
         "svdq_weight_bytes": (c_size_t, [c_int, c_int, c_int]),
         "svdq_act_bytes": (c_size_t, [c_int, c_int, c_int]),
         "svdq_weight_bytes_tiled": (c_size_t, [c_int, c_int, c_int, c_int]),
@@ -315,6 +316,26 @@ def gemm_swiglu_quant(act: QuantizedAct, w: PackedWeight, bias, w_next: PackedWe
         _check("svdq_gemm_swiglu_quant", lib().svdq_gemm_swiglu_quant(
             byref(act.desc), byref(w.desc), _ptr(bias), byref(w_next.desc), _ptr(g_x_next), byref(act_next.desc),
             _ptr(scratch), scratch.numel(), _ptr(h_out), _stream(act.device)))
+    return act_next
+
+
+def gemm_swiglu_quant_noscratch(act: QuantizedAct, w: PackedWeight, bias, w_next: PackedWeight,
+                                g_x_next: torch.Tensor, act_next: QuantizedAct,
+                                h_out: torch.Tensor | None = None) -> QuantizedAct:
+    """gemm_swiglu_quant for callers that cannot allocate: the partial sums of U' go to the
+    library's built-in 8 MiB device buffer instead of a scratch tensor (nothing is allocated here or
+    in the library). Calls on one device share that buffer: keep them ordered on one stream."""
+    if not w.swiglu:
+        raise ValueError("the gate/up weight must be packed with swiglu=True")
+    _need(g_x_next, torch.float32, "g_x_next")
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias", 1)
+    if h_out is not None:
+        _need(h_out, torch.bfloat16, "h_out", 2)
+    with torch.cuda.device(act.device):
+        _check("svdq_gemm_swiglu_quant_noscratch", lib().svdq_gemm_swiglu_quant_noscratch(
+            byref(act.desc), byref(w.desc), _ptr(bias), byref(w_next.desc), _ptr(g_x_next), byref(act_next.desc),
+            _ptr(h_out), _stream(act.device)))
     return act_next
 
 

@@ -1247,3 +1247,65 @@ svdq_status svdq_gemm_swiglu_quant(const svdq_act* act, const svdq_weight* w, co
 
 }  // extern "C"
 
+
+// ================================================================== MLP chain without caller scratch
+// svdq_gemm_swiglu_quant needs a scratch buffer for the column-split partial sums of U'. Some
+// callers have none to lend and cannot allocate one; this entry point serves them from a buffer
+// that lives in the library's own device image: a file-scope array of fixed size that every GPU
+// which loads the library holds until the process exits. In host code the array's name is only a
+// host-side stand-in, so its device address is looked up once per device (cudaGetSymbolAddress,
+// with that device current) and handed to the kernels like any caller's scratch pointer.
+namespace {
+
+constexpr size_t kMlpBuiltinScratchBytes = SVDQ_MLP_BUILTIN_SCRATCH_BYTES;  // 8 MiB
+static __device__ __align__(256) unsigned char g_mlp_builtin_scratch[kMlpBuiltinScratchBytes];
+
+struct BuiltinScratchState {
+  bool ready = false;
+  void* ptr = nullptr;
+};
+BuiltinScratchState g_builtin_scratch[64];
+
+// The device address of g_mlp_builtin_scratch on the current device (looked up on first use).
+svdq_status builtin_scratch_ptr(void** out) {
+  int dev = 0;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(SVDQ_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  BuiltinScratchState& st = g_builtin_scratch[dev];
+  if (!st.ready) {
+    void* p = nullptr;
+    SVDQ_CUDA(cudaGetSymbolAddress(&p, g_mlp_builtin_scratch));
+    if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 255u) != 0)
+      return fail(SVDQ_ERR_CUDA, "built-in scratch has no usable device address");
+    st.ptr = p;
+    st.ready = true;
+  }
+  *out = st.ptr;
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+svdq_status svdq_gemm_swiglu_quant_noscratch(const svdq_act* act, const svdq_weight* w, const uint16_t* bias,
+                                             const svdq_weight* w_next, const float* g_x_next,
+                                             const svdq_act* act_next, uint16_t* H, svdq_stream_t stream) {
+  if (act == nullptr || w == nullptr || w_next == nullptr || g_x_next == nullptr || act_next == nullptr)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const size_t need = svdq_mlp_scratch_bytes(act->M, w_next->r);
+  if (need == 0)
+    return fail(SVDQ_ERR_UNSUPPORTED, "M=%d with next-layer rank %d unsupported", act->M, w_next->r);
+  if (need > kMlpBuiltinScratchBytes)
+    return fail(SVDQ_ERR_UNSUPPORTED,
+                "M=%d at next-layer rank %d needs %zu bytes of scratch, more than the %zu-byte built-in buffer; "
+                "pass a buffer to svdq_gemm_swiglu_quant instead",
+                act->M, w_next->r, need, kMlpBuiltinScratchBytes);
+  void* scratch = nullptr;
+  if (svdq_status s = builtin_scratch_ptr(&scratch); s != SVDQ_OK) return s;
+  return svdq_gemm_swiglu_quant(act, w, bias, w_next, g_x_next, act_next, scratch, kMlpBuiltinScratchBytes, H,
+                                stream);
+}
+
+}  // extern "C"

@@ -272,6 +272,28 @@ SVDQ_API svdq_status svdq_gemm_swiglu_quant(const svdq_act* act, const svdq_weig
                                    const svdq_act* act_next, void* scratch, size_t scratch_bytes,
                                    uint16_t* H, svdq_stream_t stream);
 
+/* The same call for callers that cannot allocate device memory and have no scratch buffer to lend:
+ * a plug-in that runs inside a host framework which owns every device allocation (its enqueue step
+ * may not call cudaMalloc), or latency-bound code for which cudaMalloc's implicit device
+ * synchronisation is not acceptable. The pages have no counterpart; this is a convenience of this
+ * library. Arguments as for svdq_gemm_swiglu_quant without `scratch` / `scratch_bytes`: the
+ * partial sums go to a buffer of SVDQ_MLP_BUILTIN_SCRATCH_BYTES (8 MiB) that is part of the
+ * library's device image, so every GPU that loads the library holds it until the process exits.
+ *   - Limit: svdq_mlp_scratch_bytes(M, r_next) must not exceed that size (at r_next = 32: M <= 8192
+ *     tokens; r_next = 16: 16384; r_next = 64: 4096); larger calls return SVDQ_ERR_UNSUPPORTED and
+ *     enqueue nothing.
+ *   - The first call on a device looks up the buffer's device address (cudaGetSymbolAddress, on the
+ *     current device) and sets the kernels up; make that first call before any stream capture.
+ *   - Every call on a device uses the same buffer and leaves its contents behind (every entry a call
+ *     reads is written by the same call first). Calls whose work overlaps on the GPU -- on two
+ *     streams, or on two threads -- race on it; order them on one stream.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+#define SVDQ_MLP_BUILTIN_SCRATCH_BYTES ((size_t)8 << 20)
+SVDQ_API svdq_status svdq_gemm_swiglu_quant_noscratch(const svdq_act* act, const svdq_weight* w,
+                                                      const uint16_t* bias, const svdq_weight* w_next,
+                                                      const float* g_x_next, const svdq_act* act_next,
+                                                      uint16_t* H, svdq_stream_t stream);
+
 SVDQ_API const char* svdq_status_str(svdq_status s);
 SVDQ_API const char* svdq_last_error(void);
 SVDQ_API int svdq_abi_version(void);
