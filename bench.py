@@ -43,6 +43,8 @@ FLUSH_BYTES = 256 << 20
 # profiles/svdq_gemm_kernel_qkv2048.md, keyed by a hash of the kernel source it was taken on; any
 # change to the kernel source makes the figure stale and it is reported as null.
 PROFILED_GEMM_TRAFFIC = {("qkv_2048", "e139ca2d2d9b"): 320.76e6}
+# The same for kernel 1 (profiles/quant_act_kernel_qkv2048.md), keyed by a hash of its source.
+PROFILED_K1_TRAFFIC = {}
 
 
 def read_peaks():
@@ -58,7 +60,7 @@ def read_peaks():
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while the timed region runs (read-only)."""
 
-    def __init__(self, index: int, period_s: float = 0.01):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.index, self.period, self.samples, self.reasons = index, period_s, [], set()
         self.max_mhz = None
         self._stop = threading.Event()
@@ -116,6 +118,15 @@ def gemm_source_hash() -> str:
     return h.hexdigest()[:12]
 
 
+def k1_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("svdq_quant.cuh", "svdq_ptx.cuh"):
+        with open(os.path.join(ROOT, "bit_diffusion_transformer_svdquant_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
 def max_over_ranks(value: float, device) -> float:
     """Largest value over all ranks (the slowest replica sets the time)."""
     if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
@@ -126,7 +137,14 @@ def max_over_ranks(value: float, device) -> float:
 
 
 def layer_flops(spec):
+    """(2MNK, 2Mr(K+N)): the FP4 contraction and the whole low-rank branch (down- and up-projection)."""
     return 2.0 * spec.M * spec.N * spec.K, 2.0 * spec.M * spec.r * (spec.K + spec.N)
+
+
+def gemm_kernel_flops(spec):
+    """Method FLOPs inside the GEMM kernel: the FP4 contraction 2MNK plus the branch's up-projection
+    2MrN (the down-projection 2MKr runs in kernel 1)."""
+    return 2.0 * spec.M * spec.N * spec.K + 2.0 * spec.M * spec.r * spec.N
 
 
 def kernel1_bytes(spec):
@@ -231,13 +249,19 @@ def gpu_arm(args, rank, world, dev):
 
     K = args.steps
     n_l = len(layers)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    mids = [[torch.cuda.Event(enable_timing=True) for _ in range(n_l)] for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    # kernel-level events: quantize (kernel 1) and GEMM (kernel 2) of every layer
-    k_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-              torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(n_l)] for _ in range(K)]
+    # Events per step: one at the start, then one after each kernel (the start of the next kernel
+    # is the end of the previous one). Every timing event on the stream costs a few microseconds
+    # of drain before the next launch (measured on B200), so no redundant ones are recorded.
+    # ev[s][0] = step start; per layer i: [1 + 3i] after the amax pass (dynamic mode only, else
+    # the same event as the layer start), [2 + 3i] after kernel 1, [3 + 3i] after the GEMM.
+    def new_ev():
+        return torch.cuda.Event(enable_timing=True)
+    ev = []
+    for _ in range(K):
+        row = [new_ev()]
+        for _ in range(n_l):
+            row += [new_ev() if dyn else None, new_ev(), new_ev()]
+        ev.append(row)
 
     if world > 1:
         torch.distributed.barrier()
@@ -246,18 +270,16 @@ def gpu_arm(args, rank, world, dev):
         t_wall = time.perf_counter()
         for s in range(K):
             flush_l2(flush, clean)
-            starts[s].record(stream)
+            row = ev[s]
+            row[0].record(stream)
             for i, L in enumerate(layers):
-                ec, e0, e1, e2 = k_ev[s][i]
-                ec.record(stream)
                 if dyn:
                     svdq.calibrate_act(L["X"], L["w"], out=L["g_x"])
-                e0.record(stream)
+                    row[1 + 3 * i].record(stream)
                 svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
-                e1.record(stream)
+                row[2 + 3 * i].record(stream)
                 svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
-                e2.record(stream)
-            ends[s].record(stream)
+                row[3 + 3 * i].record(stream)
         torch.cuda.synchronize(dev)
         t_wall = time.perf_counter() - t_wall
     if world > 1:
@@ -265,11 +287,18 @@ def gpu_arm(args, rank, world, dev):
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out during the timed region")
 
-    step_ms = [starts[s].elapsed_time(ends[s]) for s in range(K)]
+    def layer_start(row, i):
+        return row[0] if i == 0 else row[3 * i]
+
+    def k1_start(row, i):
+        return row[1 + 3 * i] if dyn else layer_start(row, i)
+
+    step_ms = [ev[s][0].elapsed_time(ev[s][3 * n_l]) for s in range(K)]
     total_ms = float(sum(step_ms))
-    kc_ms = [[k_ev[s][i][0].elapsed_time(k_ev[s][i][1]) for s in range(K)] for i in range(n_l)]
-    k1_ms = [[k_ev[s][i][1].elapsed_time(k_ev[s][i][2]) for s in range(K)] for i in range(n_l)]
-    k2_ms = [[k_ev[s][i][2].elapsed_time(k_ev[s][i][3]) for s in range(K)] for i in range(n_l)]
+    kc_ms = [[layer_start(ev[s], i).elapsed_time(ev[s][1 + 3 * i]) if dyn else 0.0 for s in range(K)]
+             for i in range(n_l)]
+    k1_ms = [[k1_start(ev[s], i).elapsed_time(ev[s][2 + 3 * i]) for s in range(K)] for i in range(n_l)]
+    k2_ms = [[ev[s][2 + 3 * i].elapsed_time(ev[s][3 + 3 * i]) for s in range(K)] for i in range(n_l)]
     total_ms = max_over_ranks(total_ms, dev)
 
     flops_main = sum(layer_flops(L["spec"])[0] for L in layers)
@@ -284,10 +313,11 @@ def gpu_arm(args, rank, world, dev):
     k2_avg = statistics.mean(k2_ms[big])
     peaks = read_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
-    gemm_flops = sum(layer_flops(spec_b))
+    gemm_flops = gemm_kernel_flops(spec_b)
     achieved = gemm_flops / (k2_avg * 1e-3) / 1e12
     k1_avg = [statistics.mean(k1_ms[i]) for i in range(n_l)]
     k1_gbs = [kernel1_bytes(layers[i]["spec"]) / (k1_avg[i] * 1e-3) / 1e9 for i in range(n_l)]
+    big1 = max(range(n_l), key=lambda i: kernel1_bytes(layers[i]["spec"]))
 
     e2e = e2e_arm(args, layers, dev, world)
 
@@ -343,6 +373,14 @@ def gpu_arm(args, rank, world, dev):
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_PER_BF16}"
                                     " (nominal dense FP4/bf16 ratio)",
                      "algorithmic": f"{gemm_flops / 1e9:.1f} GFLOP per launch (2MNK + 2MrN)"},
+        "roofline_kernel1": {"bound": "hbm", "kernel": "quant_act_kernel", "achieved": round(k1_gbs[big1], 1),
+                             "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+                             "frac": round(k1_gbs[big1] / peaks["hbm_gbs"], 4),
+                             "traffic": PROFILED_K1_TRAFFIC.get((wl.name, k1_source_hash())),
+                             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                             "peak_source": f"{peaks['source']} HBM copy bandwidth",
+                             "algorithmic": f"{kernel1_bytes(layers[big1]['spec']) / 1e6:.1f} MB per launch "
+                                            "(2MK + MK/2 + MK/16 + 4Mr: X read; codes, scales, U hi/lo written)"},
         "e2e": e2e,
         "cuda_graph": {"value": round(world * flops_main / (graph_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                        "ms_per_step": round(graph_ms, 5), "steps": side_steps,
@@ -359,35 +397,91 @@ def gpu_arm(args, rank, world, dev):
     return out
 
 
+E2E_CHUNKS = 8
+
+
 def e2e_arm(args, layers, dev, world):
-    """The same metric through the public API with host buffers: every step copies the first layer's
-    X from pinned host memory, runs the layer(s), and copies the last output back to pinned host."""
+    """The same metric through the public API with host buffers: every step copies the first
+    layer's X from pinned host memory, runs the layer(s) and copies the last layer's output back to
+    pinned host memory. The layer is row-independent and its activation scale static, so the step
+    runs as E2E_CHUNKS row chunks (each a normal library call on its rows) in a three-stream
+    pipeline: the host-to-device copy of chunk i+1 and the device-to-host copy of chunk i-1 overlap
+    the kernels of chunk i (PCIe is full duplex). Timed with CUDA events on the default stream,
+    which waits for the last copy of every step."""
     import bit_diffusion_transformer_svdquant_b200 as svdq
     stream = torch.cuda.current_stream(dev)
-    X_host = layers[0]["X"].cpu().pin_memory()
+    M = layers[0]["spec"].M
+    X_dev = layers[0]["X"]
+    X_host = X_dev.cpu().pin_memory()
     Y_last = layers[-1]["Y"]
     Y_host = torch.empty(Y_last.shape, dtype=Y_last.dtype).pin_memory()
+    # row chunks on 128-row boundaries
+    step_rows = -(-M // (E2E_CHUNKS * 128)) * 128
+    bounds = [(r0, min(M, r0 + step_rows)) for r0 in range(0, M, step_rows)]
+    acts = [[svdq.QuantizedAct(r1 - r0, L["spec"].K, L["spec"].r, dev) for L in layers] for r0, r1 in bounds]
+    s_h2d, s_cmp, s_d2h = (torch.cuda.Stream(dev) for _ in range(3))
+    n = len(bounds)
+    ev_h = [torch.cuda.Event() for _ in range(n)]
+    ev_c = [torch.cuda.Event() for _ in range(n)]
+    ev_d = [torch.cuda.Event() for _ in range(n)]
+    first = [True]
+
+    def step():
+        for s_ in (s_h2d, s_cmp, s_d2h):
+            s_.wait_stream(stream)
+        for i, (r0, r1) in enumerate(bounds):
+            with torch.cuda.stream(s_h2d):
+                if not first[0]:
+                    s_h2d.wait_event(ev_c[i])       # the previous step's kernels have read X rows i
+                X_dev[r0:r1].copy_(X_host[r0:r1], non_blocking=True)
+                ev_h[i].record(s_h2d)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_h[i])
+                if not first[0]:
+                    s_cmp.wait_event(ev_d[i])       # the previous step's copy has read Y rows i
+                x = X_dev[r0:r1]
+                for L, a in zip(layers, acts[i]):
+                    svdq.quantize_act(x, L["w"], L["g_x"], a)
+                    x = svdq.gemm(a, L["w"], L["bias"], out=L["Y"][r0:r1])
+                ev_c[i].record(s_cmp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_c[i])
+                Y_host[r0:r1].copy_(Y_last[r0:r1], non_blocking=True)
+                ev_d[i].record(s_d2h)
+        first[0] = False
+        for s_ in (s_h2d, s_cmp, s_d2h):
+            stream.wait_stream(s_)
+
+    if args.dynamic_scale:
+        raise ValueError("the pipelined end-to-end leg needs a static activation scale")
     steps = max(3, min(args.steps, 20))
     for _ in range(2):
-        layers[0]["X"].copy_(X_host, non_blocking=True)
-        run_step(layers, dynamic=args.dynamic_scale)
-        Y_host.copy_(Y_last, non_blocking=True)
+        step()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
-        layers[0]["X"].copy_(X_host, non_blocking=True)
-        run_step(layers, dynamic=args.dynamic_scale)
-        Y_host.copy_(Y_last, non_blocking=True)
+        step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / steps
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out in the end-to-end loop")
+    # the pipelined result against the resident whole-M call (chunks may split kernel 1's K range
+    # differently, which changes U's fp32 summation order, so this is a difference, not equality)
+    for L in layers:
+        svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
+        svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
+    torch.cuda.synchronize(dev)
+    ref = Y_last.float().cpu()
+    rel = float((Y_host.float() - ref).abs().max() / ref.abs().max())
     flops = sum(layer_flops(L["spec"])[0] for L in layers)
     return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": X_host.numel() * X_host.element_size(),
-            "d2h_bytes_per_step": Y_host.numel() * Y_host.element_size()}
+            "d2h_bytes_per_step": Y_host.numel() * Y_host.element_size(), "chunks": n,
+            "max_rel_diff_vs_resident": rel,
+            "what": f"pinned host X -> device -> layer(s) -> pinned host Y, {n} row chunks pipelined over "
+                    "three streams (copy in, kernels, copy out)"}
 
 
 # ---------------------------------------------------------------------------------- row-wise FP8 variant
@@ -542,8 +636,20 @@ def mlp_fused_arm(args, dev):
         raise RuntimeError("device wait ran out in the fused timed region")
     ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
     part = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(3)]
+    # the unfused chain (kernel 1 + GEMM per layer, h through HBM) under the same protocol
+    unf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for s in range(K):
+        flush_l2(flush, clean)
+        unf[s][0].record(stream)
+        run_step([up, dn])
+        unf[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out in the unfused timed region")
+    ms_unf = statistics.mean(a.elapsed_time(b) for a, b in unf)
     flops = layer_flops(up["spec"])[0] + layer_flops(dn["spec"])[0]
     return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+            "unfused_ms_per_step": round(ms_unf, 5), "saving_us": round((ms_unf - ms) * 1e3, 2),
             "steps": K, "warmup": args.warmup,
             "kernels_us": {"quantize_act_up": round(part[0] * 1e3, 2), "gemm_swiglu_quant": round(part[1] * 1e3, 2),
                            "gemm_down": round(part[2] * 1e3, 2)},
@@ -552,10 +658,66 @@ def mlp_fused_arm(args, dev):
                     "GEMM; run in a separate process"}
 
 
-def child_side(args, flag):
+def config_row_arm(args, dev):
+    """Compact figures of one workload under the main protocol (write-flush between steps, CUDA
+    events): the side table of the other workloads in the default line."""
+    import bit_diffusion_transformer_svdquant_b200 as svdq
+    wl = synth.WORKLOADS[args.workload]
+    layers = build_layers(wl, dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        run_step(layers)
+    torch.cuda.synchronize(dev)
+    K, n_l = args.steps, len(layers)
+    ev = [[tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_l)] for _ in range(K)]
+    for s_ in range(K):
+        flush_l2(flush)
+        for i, L in enumerate(layers):
+            e0, e1, e2 = ev[s_][i]
+            e0.record(stream)
+            svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
+            e1.record(stream)
+            svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
+            e2.record(stream)
+    torch.cuda.synchronize(dev)
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out")
+    ms = statistics.mean(ev[s_][0][0].elapsed_time(ev[s_][-1][2]) for s_ in range(K))
+    k1 = [statistics.mean(ev[s_][i][0].elapsed_time(ev[s_][i][1]) for s_ in range(K)) for i in range(n_l)]
+    k2 = [statistics.mean(ev[s_][i][1].elapsed_time(ev[s_][i][2]) for s_ in range(K)) for i in range(n_l)]
+    peaks = read_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    flops = sum(layer_flops(L["spec"])[0] for L in layers)
+    value = flops / (ms * 1e-3) / 1e12
+    return {"value": round(value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+            "frac_fp4_peak_e2e": round(value / fp4_peak, 4),
+            "tokens_per_s": round(layers[0]["spec"].M / (ms * 1e-3), 1),
+            "quantize_act_us": [round(x * 1e3, 2) for x in k1],
+            "quantize_act_frac_hbm": [round(kernel1_bytes(L["spec"]) / (x * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+                                      for L, x in zip(layers, k1)],
+            "gemm_us": [round(x * 1e3, 2) for x in k2],
+            "gemm_frac_fp4_peak": [round(gemm_kernel_flops(L["spec"]) / (x * 1e-3) / 1e12 / fp4_peak, 4)
+                                   for L, x in zip(layers, k2)],
+            "steps": K}
+
+
+SIDE_WORKLOADS = ("tiny", "qkv_1024", "mlp_1024", "edit_2048")
+
+
+def configs_side(args):
+    """config_row_arm for every other workload, each in a child process."""
+    out = {}
+    for name in SIDE_WORKLOADS:
+        if name != args.workload:
+            out[name] = child_side(args, "--config-row-only", workload=name)
+    return out
+
+
+def child_side(args, flag, workload=None):
     """An arm of this script in a child process (its own CUDA context and a time limit), so that
     nothing in it can affect the main measurement; any failure comes back as {"error": ...}."""
-    cmd = [sys.executable, os.path.abspath(__file__), flag, "--workload", args.workload,
+    cmd = [sys.executable, os.path.abspath(__file__), flag, "--workload", workload or args.workload,
            "--steps", str(max(3, min(args.steps, 50))), "--warmup", "3"] + (["--l2-clean"] if getattr(args, "l2_clean", False) else [])
     try:
         r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
@@ -678,6 +840,9 @@ def main():
                     help="after each 256 MB write-flush also read 256 MB, so steps start with clean L2 lines")
     ap.add_argument("--fp8r-only", action="store_true", help=argparse.SUPPRESS)
     ap.add_argument("--mlp-fused-only", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--config-row-only", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--no-side-configs", action="store_true",
+                    help="skip the side table of the other workloads")
     ap.add_argument("--no-mlp-fused", action="store_true",
                     help="skip the fused-chain side measurement of the MLP workloads")
     args = ap.parse_args()
@@ -701,6 +866,9 @@ def main():
     if args.mlp_fused_only:
         print(json.dumps(mlp_fused_arm(args, dev)), flush=True)
         return
+    if args.config_row_only:
+        print(json.dumps(config_row_arm(args, dev)), flush=True)
+        return
     if world > 1:
         from datetime import timedelta
         torch.distributed.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
@@ -709,8 +877,13 @@ def main():
         if rank == 0:
             if world == 1 and not args.no_fp8r:
                 out["fp8r_variant"] = fp8r_side(args)
-            if world == 1 and args.workload.startswith("mlp") and not args.no_mlp_fused:
-                out["mlp_fused"] = child_side(args, "--mlp-fused-only")
+            if world == 1 and not args.no_mlp_fused:
+                # the MLP chain with the down layer's kernel 1 fused, on this workload if it is an
+                # MLP, else on the 1024^2 MLP
+                mlp_wl = args.workload if args.workload.startswith("mlp") else "mlp_1024"
+                out["mlp_fused"] = {"workload": mlp_wl, **child_side(args, "--mlp-fused-only", workload=mlp_wl)}
+            if world == 1 and not args.no_side_configs:
+                out["configs"] = configs_side(args)
             if world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
             print(json.dumps(out), flush=True)

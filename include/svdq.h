@@ -266,7 +266,8 @@ SVDQ_API size_t svdq_mlp_scratch_bytes(int M, int r_next);
  *                 are bit-identical to that path, U agrees to fp32 summation order
  *   scratch       device, >= svdq_mlp_scratch_bytes(M, r_next), 16-byte aligned
  *   H             optional device bf16 [M][N/2] that also receives h (NULL: h is not stored)
- * Not captured by any GPU parity record yet. */
+ * GPU tests check the down layer's codes, scales and alpha bit-exactly and its output within 2e-3
+ * against the oracle on the h this call produced, and against the unfused two-call chain. */
 SVDQ_API svdq_status svdq_gemm_swiglu_quant(const svdq_act* act, const svdq_weight* w, const uint16_t* bias,
                                    const svdq_weight* w_next, const float* g_x_next,
                                    const svdq_act* act_next, void* scratch, size_t scratch_bytes,
