@@ -49,6 +49,7 @@ struct DeviceState {
   bool ready = false;
   int sm_count = 0;
   int max_pairs[3] = {0, 0, 0};  // co-resident CTA pairs of the GEMM kernel for n_tile 256, 192, 128
+  int k1_clusters[4][3] = {};     // co-resident kernel-1 clusters, by r (0/16/32/64) and size (1/2/4)
   svdq_status status = SVDQ_OK;
   std::string error;
 };
@@ -96,13 +97,13 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<128, kStagesTile128>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<0>::kSmem));
+                                   svdq::Q1Layout<0>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<16>::kSmem));
+                                   svdq::Q1Layout<16>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<32>::kSmem));
+                                   svdq::Q1Layout<32>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<64>::kSmem));
+                                   svdq::Q1Layout<64>::kSmem));
     // How many CTA pairs of each GEMM instantiation can be resident at once: the persistent grid
     // never asks for more (pairs must sit on two SMs of one GPC, so this can be below sms / 2).
     auto max_pairs = [&](const void* fn, int smem, int* out) -> svdq_status {
@@ -126,6 +127,43 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
       return s;
     if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::svdq_gemm_kernel<128, kStagesTile128>),
                                   svdq::GemmLayout<128, kStagesTile128>::kSmem, &st.max_pairs[2]);
+        s != SVDQ_OK)
+      return s;
+    // how many kernel-1 clusters of 1, 2 and 4 CTAs (one CTA per SM) can be resident at once
+    auto k1_clusters = [&](const void* fn, int smem, int* out) -> svdq_status {
+      for (int ci = 0; ci < 3; ++ci) {
+        const int c = 1 << ci;
+        cudaLaunchConfig_t cfg{};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(c * (sms / c), 1, 1);
+        cfg.blockDim = dim3(svdq::kQ1Threads, 1, 1);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, fn, &cfg));
+        out[ci] = n;
+      }
+      return SVDQ_OK;
+    };
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<0>), svdq::Q1Layout<0>::kSmem,
+                                    st.k1_clusters[0]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<16>),
+                                    svdq::Q1Layout<16>::kSmem, st.k1_clusters[1]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<32>),
+                                    svdq::Q1Layout<32>::kSmem, st.k1_clusters[2]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<64>),
+                                    svdq::Q1Layout<64>::kSmem, st.k1_clusters[3]);
         s != SVDQ_OK)
       return s;
     st.sm_count = sms;
@@ -458,15 +496,18 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
         s != SVDQ_OK)
       return s;
   }
-  // K split across a cluster of 1, 2 or 4 CTAs so that small M still fills the SMs. Measured on
-  // B200 (K = 3072, r = 32): pairs beat single CTAs at 36 and 132 row tiles (38 vs 54 us, 52 vs
-  // 60 us) and clusters of 4 (45 and 95 us: fewer clusters of 4 are co-resident). Clusters of 4
-  // only for a handful of row tiles. SVDQ_K1_CLUSTER overrides the size; every CTA keeps whole
-  // 64-column K steps.
+  // One CTA per SM; K is split across a cluster of 2 or 4 CTAs only while all row tiles' clusters
+  // of that size are resident at once (cudaOccupancyMaxActiveClusters: clusters must fit inside
+  // GPCs), so small M fills more SMs and nothing runs as a second wave. SVDQ_K1_CLUSTER overrides
+  // the size; every CTA keeps whole 64-column K steps.
   const int m_tiles = act->M_pad / 128;
   int csize = 1;
-  if (m_tiles < 2 * sms && (K / 2) % 64 == 0) csize = 2;
-  if (16 * m_tiles <= sms && (K / 4) % 64 == 0) csize = 4;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    const int* mc = g_dev[dev].k1_clusters[r == 0 ? 0 : r == 16 ? 1 : r == 32 ? 2 : 3];
+    if (m_tiles <= mc[1] && (K / 2) % 64 == 0) csize = 2;
+    if (m_tiles <= mc[2] && (K / 4) % 64 == 0) csize = 4;
+  }
   if (const char* env = getenv("SVDQ_K1_CLUSTER"); env != nullptr) {
     const int c = atoi(env);
     if ((c == 1 || c == 2 || c == 4) && (K / c) % 64 == 0) csize = c;
@@ -492,26 +533,26 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(m_tiles * csize, 1, 1);
-  cfg.blockDim = dim3(svdq::kQThreads, 1, 1);
+  cfg.blockDim = dim3(svdq::kQ1Threads, 1, 1);
   cfg.stream = static_cast<cudaStream_t>(stream);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaSuccess;
   switch (r) {
     case 0:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<0>::kSmem;
+      cfg.dynamicSmemBytes = svdq::Q1Layout<0>::kSmem;
       e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<0>, tmX, tmL1, a);
       break;
     case 16:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<16>::kSmem;
+      cfg.dynamicSmemBytes = svdq::Q1Layout<16>::kSmem;
       e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<16>, tmX, tmL1, a);
       break;
     case 32:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<32>::kSmem;
+      cfg.dynamicSmemBytes = svdq::Q1Layout<32>::kSmem;
       e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<32>, tmX, tmL1, a);
       break;
     case 64:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<64>::kSmem;
+      cfg.dynamicSmemBytes = svdq::Q1Layout<64>::kSmem;
       e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<64>, tmX, tmL1, a);
       break;
     default: return fail(SVDQ_ERR_UNSUPPORTED, "r=%d unsupported", r);

@@ -83,8 +83,8 @@ struct GemmLayout {
   static constexpr int kStageOutWarp = 4096;
   static constexpr int kOutOff = STAGES * kStage;
   static constexpr int kBarOff = kOutOff + 8 * kStageOutWarp;
-  // full[STAGES], empty[STAGES], accf[kAccBufs], acce[kAccBufs], drain, sf_full[kSfBufs]
-  static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1 + kSfBufs;
+  // full[STAGES], empty[STAGES], sf_land[STAGES], accf[kAccBufs], acce[kAccBufs], drain, sf_full[kSfBufs]
+  static constexpr int kNumBars = 3 * STAGES + 2 * kAccBufs + 1 + kSfBufs;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kColSf + kSfBufs * kSfCols <= 512, "TMEM budget");
@@ -147,12 +147,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + L::kBarOff;
+  // full: in the even CTA, the A / B (or low-rank) bytes of both CTAs of a ring slot (the pair
+  // loads complete there); sf_land: this CTA's scale-factor bytes of a slot
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
-  auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + kAccBufs + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * kAccBufs);
-  auto sf_full_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * kAccBufs + 1 + b); };
+  auto sf_land_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + kAccBufs + b); };
+  const uint32_t drain_bar = bar0 + 8u * (3 * STAGES + 2 * kAccBufs);
+  auto sf_full_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + 2 * kAccBufs + 1 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -163,8 +166,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), 1);   // the even CTA's producer arrives (with both CTAs' byte count)
       mbar_init(empty_bar(s), 1);
+      mbar_init(sf_land_bar(s), 1);
     }
     for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(accf_bar(b), 1);
@@ -197,11 +201,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // Per ring slot: this CTA's scale atoms (1-D bulk copies onto its own sf_land barrier, first,
+      // so that the writers can store them while A and B are still in flight), then its 128 A rows
+      // and n_tile/2 B rows as CTA-pair TMA loads that complete on the even CTA's full barrier; the
+      // even CTA's producer expects the bytes of both CTAs there.
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       const int rc = r < kLrChunk ? r : kLrChunk;
       const uint32_t lr_bytes = static_cast<uint32_t>((2 * 128 + L::kBRows) * rc * 2);
       const int sf_row_stride = args.K >> 6;  // 64-wide K atoms per 128-row block
+      const bool leader = rank == 0;
       bool ok = true;
       for (int tile = pair0; ok && tile < args.num_tiles; tile += npairs) {
         int m_pair, n_blk;
@@ -215,10 +224,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
             break;
           const uint32_t sa = sbase + stage * L::kStage;
-          mbar_arrive_expect_tx(full_bar(stage), lr_bytes);
-          tma_load_2d(sa, &tmU, c0, m_blk * 128, full_bar(stage));
-          tma_load_2d(sa + kOffULo, &tmU, c0, args.M_pad + m_blk * 128, full_bar(stage));
-          tma_load_2d(sa + L::kOffB, &tmL2, c0, b_row, full_bar(stage));
+          mbar_arrive(sf_land_bar(stage));  // no scales in a low-rank slot: its sf_land phase completes now
+          const uint32_t fb = cluster_map(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * lr_bytes);
+          tma_load_2d_pair(sa, &tmU, c0, m_blk * 128, fb);
+          tma_load_2d_pair(sa + kOffULo, &tmU, c0, args.M_pad + m_blk * 128, fb);
+          tma_load_2d_pair(sa + L::kOffB, &tmL2, c0, b_row, fb);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -230,21 +241,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
             break;
           const uint32_t sa = sbase + stage * L::kStage;
-          mbar_arrive_expect_tx(full_bar(stage), L::kStage);
-          tma_load_2d(sa, &tmA, kt * 128, m_blk * 128, full_bar(stage));
-          tma_load_2d(sa + L::kOffB, &tmB, kt * 128, b_row, full_bar(stage));
-          bulk_load(sa + L::kOffSfa, sfa_tile + (static_cast<size_t>(kt) * 4 << 9), L::kSfa, full_bar(stage));
+          mbar_arrive_expect_tx(sf_land_bar(stage), L::kSfa + L::kSfb);
+          bulk_load(sa + L::kOffSfa, sfa_tile + (static_cast<size_t>(kt) * 4 << 9), L::kSfa, sf_land_bar(stage));
           bulk_load(sa + L::kOffSfb, sfb_tile + (static_cast<size_t>(kt) * 4 * L::kSfAtomsB << 9), L::kSfb,
-                    full_bar(stage));
+                    sf_land_bar(stage));
+          const uint32_t fb = cluster_map(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * (L::kA + L::kB));
+          tma_load_2d_pair(sa, &tmA, kt * 128, m_blk * 128, fb);
+          tma_load_2d_pair(sa + L::kOffB, &tmB, kt * 128, b_row, fb);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      // Drain: every copy this thread started has landed before the CTA may exit.
+      // Drain: every copy this thread started has landed before the CTA may exit. A slot's release
+      // (its MMAs have read it, so all its copies landed) shows it; after an abort the bounded
+      // wait's limit, far longer than any copy takes, does.
       for (int s = 0; s < STAGES; ++s)
         if (armed & (1u << s))
-          mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
+          mbar_wait_bounded(empty_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
@@ -256,8 +271,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // B200. The whole warp runs this loop (warp-uniform operands); elect.sync inside the MMA and
     // commit helpers picks the issuing lane, and a wait succeeds only when it succeeds in every lane.
     if (rank == 0) {
-      auto wait_all = [&](uint32_t bar, uint32_t parity, unsigned code, volatile int* abort_ptr) {
-        return __all_sync(0xffffffffu, mbar_wait_bounded_cluster(bar, parity, wait_ns, status, code, abort_ptr));
+      auto wait_all = [&](uint32_t bar, uint32_t parity, unsigned code, volatile int* abort_ptr) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait_bounded_cluster(bar, parity, wait_ns, status, code, abort_ptr)) != 0;
+      };
+      // the slot's A / B (or low-rank) bytes of both CTAs, then its scale buffer (both CTAs' writers)
+      auto wait_slot = [&](int stage_, uint32_t phase_, int sfb_, uint32_t sf_phase_) -> bool {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(stage_), phase_, wait_ns, status, kStatusMma,
+                                                       abort_flag)))
+          return false;
+        return wait_all(sf_full_bar(sfb_), sf_phase_, kStatusMma, abort_flag);
       };
       const int num_tiles = args.num_tiles, k_iters = args.k_iters;
       const int rc = r < kLrChunk ? r : kLrChunk;
@@ -279,7 +301,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
         uint32_t accumulate = 0;
         for (int c0 = 0; c0 < r; c0 += kLrChunk) {
-          if (!(ok = wait_all(sf_full_bar(sfb), sf_phase, kStatusMma, abort_flag))) break;
+          if (!(ok = wait_slot(stage, phase, sfb, sf_phase))) break;
           tc_fence_after();
           const uint32_t lo = lo0 + stage * (L::kStage >> 4);
           for (int j = 0; j < nj; ++j) {
@@ -294,7 +316,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         for (int kt = 0; kt < k_iters; ++kt) {
-          if (!(ok = wait_all(sf_full_bar(sfb), sf_phase, kStatusMma, abort_flag))) break;
+          if (!(ok = wait_slot(stage, phase, sfb, sf_phase))) break;
           tc_fence_after();
           const uint32_t la = lo0 + stage * (L::kStage >> 4);
           const uint32_t lb = la + (L::kOffB >> 4);
@@ -325,6 +347,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // the block-scaled MMA reads: for a 128-row atom, lane l, column c holds the 4 E4M3 scales of
     // row l + 32 c -- exactly bytes [16 l, 16 l + 16) of the 512-byte atom in shared memory. Every
     // ring slot (low-rank chunks too, which carry no scales) is reported to the issuer's barrier.
+    // The writers wait only for this CTA's scale bytes (sf_land), not for A and B, so their work
+    // overlaps the rest of the slot's copies; the issuer waits for A and B itself.
     const int q = warp & 3;
     int stage = 0, sfb = 0, slots_done = 0;
     uint32_t phase = 0;
@@ -332,7 +356,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     for (int tile = pair0; ok && tile < args.num_tiles; tile += npairs) {
       for (int slot = 0; slot < lr_slots + args.k_iters; ++slot) {
-        const bool got_data = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
+        const bool got_data = mbar_wait_bounded(sf_land_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
         if (!__all_sync(0xffffffffu, got_data)) { ok = false; break; }
         const bool has_sf = slot >= lr_slots;
         // read the stage's scale atoms now; only the TMEM stores wait for the buffer

@@ -127,31 +127,37 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
 // ------------------------------------------------------------------------------------------------
 // Kernel 1: smoothing + NVFP4 activation quantization + U = X L1s, one pass over X.
 //
-// A CTA owns 128 rows of X and a K range (a cluster of 1, 2 or 4 CTAs splits K when there are few
-// row tiles). TMA streams 128 x 64 bf16 stages (128B swizzle) of X, and 64-column slices of
-// L1s^T, into a 4-deep shared-memory ring. Every stage is read twice from shared memory: by eight
-// quantizer warps (smoothing, block amax, E4M3 scale, E2M1 codes; codes and scales go straight to
-// global memory), and by a single-thread tcgen05 bf16 MMA (M=128, N=r, K=16) that accumulates the
-// down-projection in TMEM. X thus crosses HBM once. At the end four warps read U from TMEM; with
-// a K split the partial U of every CTA is summed in rank order through distributed shared memory.
-// U is stored divided by alpha = g_x g_w (one scale for the whole GEMM) as a bf16 hi/lo pair.
-constexpr int kQThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 quantize (2..5 also drain U)
-constexpr int kQStages = 4;
+// A CTA (one per SM) owns 128 rows of X and a K range: the whole K, or a share of it when a
+// thread-block cluster of 2 or 4 CTAs splits K so that few row tiles still fill the SMs in one
+// wave. TMA streams 128 x 64 bf16 stages (128B swizzle; an L2 evict-first policy, since X is read
+// once) of X, the stage's 64-column slice of L1s^T and its 64 inverse smoothing factors into an
+// 8-deep shared-memory ring (6 at r = 64). Every stage is read twice from shared memory: by one of
+// two groups of eight quantizer warps (the groups take alternate stages, so two stages are being
+// quantized at any time: smoothing, block amax, E4M3 scale, E2M1 codes, stored straight to global
+// memory), and by a single-thread tcgen05 bf16 MMA (M=128, N=r, K=16) that accumulates the
+// down-projection in TMEM. X thus crosses HBM once. At the end four warps read U from TMEM; with a
+// K split the partial U of every CTA is summed in rank order through distributed shared memory. U
+// is stored divided by alpha = g_x g_w (one scale for the whole GEMM) as a bf16 hi/lo pair.
 constexpr int kQTile = 128 * 128;  // 128 rows x 64 bf16
+constexpr int kQuantWarps = 16;    // two groups of eight
+constexpr int kQ1Threads = 64 + 32 * kQuantWarps;  // warp 0 TMA, warp 1 MMA, warps 2..17 quantize (2..5 drain U)
 
 template <int R>
-struct QuantLayout {
+struct Q1Layout {
+  static constexpr int kStages = R <= 32 ? 8 : 6;
   static constexpr int kL1 = (R * 128 + 1023) / 1024 * 1024;
   static constexpr int kLamOff = kQTile + kL1;      // the stage's 64 inverse smoothing factors (fp32)
   static constexpr int kStage = kQTile + kL1 + 1024;
-  static constexpr int kPartOff = kQStages * kStage;
+  static constexpr int kPartOff = kStages * kStage;
   static constexpr int kPart = R * 128 * 4 + 128 * 4;  // rows padded to R + 1 floats
   static constexpr int kTabOff = kPartOff + kPart;        // 128 fp32: 1 / (dec(s) g_x) per scale code
   static constexpr int kBarOff = kTabOff + 128 * 4;
-  static constexpr int kNumBars = 2 * kQStages + 2;
+  static constexpr int kNumBars = 2 * kStages + 2;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
   static constexpr int kTmemCols = R <= 32 ? 32 : 64;
   static_assert(kStage % 1024 == 0, "stage alignment");
+  static_assert(kStages % 2 == 0, "each quantizer group owns the ring slots of one parity");
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct QuantActArgs {
@@ -167,17 +173,18 @@ struct QuantActArgs {
 };
 
 template <int R>
-__global__ void __launch_bounds__(kQThreads, 2)
+__global__ void __launch_bounds__(kQ1Threads, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL1,
                      const QuantActArgs a) {
-  using L = QuantLayout<R>;
+  using L = Q1Layout<R>;
+  constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + L::kBarOff;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kQStages + s); };
-  const uint32_t accf_bar = bar0 + 8u * (2 * kQStages);
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  const uint32_t accf_bar = bar0 + 8u * (2 * S);
   const uint32_t drain_bar = accf_bar + 8u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -192,9 +199,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
   const uint64_t wait_ns = a.wait_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 8 + (R > 0 ? 1 : 0));
+      mbar_init(empty_bar(s), 8 + (R > 0 ? 1 : 0));  // one quantizer group + the MMA commit
     }
     mbar_init(accf_bar, 1);
     mbar_init(drain_bar, 1);
@@ -221,6 +228,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
   if (warp == 0) {
     if (lane == 0) {
+      const uint64_t pol_x = l2_policy_evict_first();
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       for (int st = 0; st < n_steps; ++st) {
@@ -228,14 +236,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
         const uint32_t sa = sbase + stage * L::kStage;
         mbar_arrive_expect_tx(full_bar(stage), kQTile + R * 128 + 256);
         const int kx = kbeg + (st << 6);
-        tma_load_2d(sa, &tmX, kx, m_tile * 128, full_bar(stage));
+        tma_load_2d_hint(sa, &tmX, kx, m_tile * 128, full_bar(stage), pol_x);
         if (R > 0) tma_load_2d(sa + kQTile, &tmL1, kx, 0, full_bar(stage));
         bulk_load(sa + L::kLamOff, a.inv_lambda + kx, 256, full_bar(stage));
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+        if (++stage == S) { stage = 0; phase ^= 1u; }
       }
-      for (int s = 0; s < kQStages; ++s)
+      for (int s = 0; s < S; ++s)
         if (armed & (1u << s))
           mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
     }
@@ -257,26 +265,37 @@ __global__ void __launch_bounds__(kQThreads, 2)
           accumulate = 1;
         }
         tc_commit(empty_bar(stage));
-        if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+        if (++stage == S) { stage = 0; phase ^= 1u; }
       }
       if (ok) tc_commit(accf_bar);
       tc_commit(drain_bar);
       mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
     }
   } else {
-    // quantizers: thread t of the 256 owns 16-element block b = t % 4 of rows t / 4 and t / 4 + 64
-    // of the stage. The four threads of a row read its 128 swizzled bytes; a warp's 16-byte reads
-    // cover 8 rows x 4 blocks and stay conflict-free (chunks 2b and 2b+1 XOR row % 8).
-    const int t = threadIdx.x - 64;
+    // quantizers: group g = (warp - 2) / 8 takes stages g, g + 2, ...; within the group, thread t
+    // of 256 owns 16-element block b = t % 4 of rows t / 4 and t / 4 + 64 of the stage. The four
+    // threads of a row read its 128 swizzled bytes; a warp's 16-byte reads cover 8 rows x 4 blocks
+    // and stay conflict-free (chunks 2b and 2b+1 XOR row % 8).
+    const int qw = warp - 2;
+    const int grp = qw >> 3;
+    const int t = ((qw & 7) << 5) + lane;
     const int b = t & 3;
     const float d6 = __fmul_rn(6.0f, gx);
-    int stage = 0;
+    // this thread's code and scale destinations at step 0; each step moves 32 code bytes along the
+    // row and one 512-byte scale atom along K
+    uint8_t* code_ptr[2];
+    uint8_t* sf_ptr[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int row = m_tile * 128 + (t >> 2) + 64 * i;
+      code_ptr[i] = a.codes + static_cast<size_t>(row) * (K >> 1) + ((kbeg + (b << 4)) >> 1);
+      sf_ptr[i] = a.sf + act_sf_offset(row, (kbeg >> 4) + b, K);
+    }
+    int stage = grp;
     uint32_t phase = 0;
-    for (int st = 0; st < n_steps; ++st) {
+    for (int st = grp; st < n_steps; st += 2) {
       const bool got = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
-      const int kst = kbeg + (st << 6);
-      const int k = kst + (b << 4);
       const uint8_t* tile = smem + stage * L::kStage;
       // this thread's 16 inverse smoothing factors travelled with the stage (a broadcast read: the
       // threads of one block index b share them)
@@ -294,9 +313,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
         x[i][0] = *reinterpret_cast<const uint4*>(tile + rl * 128 + (((2 * b) ^ (rl & 7)) << 4));
         x[i][1] = *reinterpret_cast<const uint4*>(tile + rl * 128 + (((2 * b + 1) ^ (rl & 7)) << 4));
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(stage));  // the stage's data is in registers
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int rl = (t >> 2) + 64 * i;
         const uint32_t wx[8] = {x[i][0].x, x[i][0].y, x[i][0].z, x[i][0].w, x[i][1].x, x[i][1].y, x[i][1].z, x[i][1].w};
         float2 v[8];
         float amax = 0.0f;
@@ -320,20 +340,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
           codes.x = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q));
           codes.y = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q + 8));
         }
-        const int row = m_tile * 128 + rl;
-        *reinterpret_cast<uint2*>(a.codes + static_cast<size_t>(row) * (K >> 1) + (k >> 1)) = codes;
-        // the row's four block scales form one 32-bit word of the scale atom
-        const int base = (threadIdx.x & 31) & ~3;
-        const uint32_t s0 = __shfl_sync(0xffffffffu, sc, base);
-        const uint32_t s1 = __shfl_sync(0xffffffffu, sc, base + 1);
-        const uint32_t s2 = __shfl_sync(0xffffffffu, sc, base + 2);
-        const uint32_t s3 = __shfl_sync(0xffffffffu, sc, base + 3);
-        if (b == 0)
-          *reinterpret_cast<uint32_t*>(a.sf + act_sf_offset(row, kst >> 4, K)) = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        *reinterpret_cast<uint2*>(code_ptr[i] + (st << 5)) = codes;
+        sf_ptr[i][static_cast<size_t>(st) << 9] = static_cast<uint8_t>(sc);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar(stage));
-      if (++stage == kQStages) { stage = 0; phase ^= 1u; }
+      stage += 2;
+      if (stage >= S) { stage -= S; phase ^= 1u; }
     }
     if constexpr (R > 0) {
       // warps 2..5 (quadrant q = warp % 4) read this CTA's rows of U from TMEM; a lone CTA
@@ -364,11 +375,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
         } else {
 #pragma unroll
           for (int j = 0; j < R; j += 32) {
-            float t[32];
-            tmem_ld_32x32(ta + j, t);
+            float t32[32];
+            tmem_ld_32x32(ta + j, t32);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) u[j + e] = t[e];
+            for (int e = 0; e < 32; ++e) u[j + e] = t32[e];
           }
         }
         if (csize > 1 && crank != 0) {
@@ -422,6 +433,26 @@ __global__ void __launch_bounds__(kQThreads, 2)
     tmem_dealloc(tmem, L::kTmemCols);
   }
 }
+
+// The ring layout of kernel 1 as it was before the two-group rewrite, still used by the row-wise
+// FP8 variant's quantizing kernel (four stages, eight quantizer warps, two CTAs per SM).
+constexpr int kQThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 quantize (2..5 also drain U)
+constexpr int kQStages = 4;
+
+template <int R>
+struct QuantLayout {
+  static constexpr int kL1 = (R * 128 + 1023) / 1024 * 1024;
+  static constexpr int kLamOff = kQTile + kL1;
+  static constexpr int kStage = kQTile + kL1 + 1024;
+  static constexpr int kPartOff = kQStages * kStage;
+  static constexpr int kPart = R * 128 * 4 + 128 * 4;
+  static constexpr int kTabOff = kPartOff + kPart;
+  static constexpr int kBarOff = kTabOff + 128 * 4;
+  static constexpr int kNumBars = 2 * kQStages + 2;
+  static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
+  static constexpr int kTmemCols = R <= 32 ? 32 : 64;
+  static_assert(kStage % 1024 == 0, "stage alignment");
+};
 
 // ------------------------------------------------------------------------------------------------
 // Offline pack and calibration helpers.

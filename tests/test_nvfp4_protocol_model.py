@@ -2,16 +2,26 @@
 csrc/svdq_gemm.cuh), checked on the host like test_fused_protocol_model.py: producer, MMA issuer,
 the four scale-factor writer warps and the eight epilogue warps of both CTAs replay their barrier
 traffic in the kernel's order, with copies and MMA completions landing late and in random order.
+
+Protocol per ring slot: both CTAs' A / B (or low-rank) copies complete on the even CTA's full
+barrier, whose phase also needs the even producer's arrive (it expects both CTAs' bytes); each CTA's
+scale atoms complete on its own sf_land barrier (a low-rank slot's producer completes that phase at
+once); the writers wait for sf_land only, store the scales and arrive on the even CTA's sf_full;
+the issuer waits for full and sf_full, issues the MMAs and commits to both CTAs' empty barriers.
+At the end each producer waits for the release of every slot it filled, so no copy is in flight
+when its CTA exits.
+
 Both accumulator modes are covered: one 256- or 192-column buffer (5-stage ring), and two
-128-column buffers used alternately (6-stage ring), the mode whose multi-tile runs the full-size
-workloads do not reach. Checked: no deadlock, no stray arrival, waits on exactly their completion,
-no resource used before its previous user is done; removing any one wait must make it fail."""
+128-column buffers used alternately (6-stage ring). Checked: no deadlock, no stray arrival, waits on
+exactly their completion, no resource used before its previous user is done; removing any one wait
+must make it fail."""
 import random
 
 import pytest
 
 SF_BUFS = 4
-WAITS = ["producer.empty", "issuer.acce", "issuer.sf_full", "sf.full", "sf.release", "epi.accf"]
+WAITS = ["producer.empty", "producer.drain", "issuer.acce", "issuer.full", "issuer.sf_full", "sf.land",
+         "sf.release", "epi.accf"]
 
 
 class Barrier:
@@ -28,16 +38,19 @@ class Barrier:
 
 def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
     rng = random.Random(seed)
-    slots = (r + 31) // 32 + k_iters
+    lr_slots = (r + 31) // 32
+    slots = lr_slots + k_iters
     B = {}
 
     def bar(name, count):
         B[name] = Barrier(name, count)
 
+    for s in range(stages):
+        bar(f"full.{s}", 3)          # the even producer's arrive + the landing of each CTA's copies
     for c in (0, 1):
         for s in range(stages):
-            bar(f"full{c}.{s}", 1)
             bar(f"empty{c}.{s}", 1)
+            bar(f"sf_land{c}.{s}", 2)  # the producer's arrive + the landing of the scale atoms
         for a in range(acc_bufs):
             bar(f"accf{c}.{a}", 1)
     for a in range(acc_bufs):
@@ -46,6 +59,17 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
         bar(f"sf_full{b}", 8)
     done = lambda name: B[name].completed  # noqa: E731
     in_flight = []
+    issued = {c: [0] * stages for c in (0, 1)}
+    landed = {c: [0] * stages for c in (0, 1)}
+
+    def land(c, s):
+        def f():
+            landed[c][s] += 1
+            B[f"full.{s}"].arrive()
+        return f
+
+    def arrive(name):
+        return lambda: B[name].arrive()
 
     def wait(tag, name, index):
         if tag in skip:
@@ -58,12 +82,25 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
     def producer(c):
         uses = [0] * stages
         stage = 0
-        for _ in range(n_tiles * slots):
+        for g in range(n_tiles * slots):
+            has_sf = g % slots >= lr_slots
             yield from wait("producer.empty", f"empty{c}.{stage}", uses[stage] - 1)
             assert done(f"empty{c}.{stage}") >= uses[stage], "ring stage refilled while its MMAs read it"
             uses[stage] += 1
-            in_flight.append(f"full{c}.{stage}")
+            if has_sf:
+                B[f"sf_land{c}.{stage}"].arrive()
+                in_flight.append(arrive(f"sf_land{c}.{stage}"))
+            else:
+                B[f"sf_land{c}.{stage}"].arrive(2)
+            if c == 0:
+                B[f"full.{stage}"].arrive()
+            issued[c][stage] += 1
+            in_flight.append(land(c, stage))
             stage = (stage + 1) % stages
+        for s in range(stages):
+            if uses[s]:
+                yield from wait("producer.drain", f"empty{c}.{s}", uses[s] - 1)
+        assert landed[c] == issued[c], "CTA may exit with a copy in flight"
 
     def issuer():
         stage, sfb, g = 0, 0, 0
@@ -73,29 +110,40 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
             yield from wait("issuer.acce", f"acce{a}", use - 1)
             assert done(f"acce{a}") >= use, "accumulator overwritten before its epilogue read it"
             for _ in range(slots):
+                yield from wait("issuer.full", f"full.{stage}", g // stages)
                 yield from wait("issuer.sf_full", f"sf_full{sfb}", sf_uses[sfb])
                 sf_uses[sfb] += 1
                 for c in (0, 1):
-                    assert done(f"full{c}.{stage}") >= g // stages + 1, "MMA before a CTA's copy landed"
+                    assert landed[c][stage] >= g // stages + 1, "MMA before a CTA's copy landed"
+                    assert stored[c][g] if g < len(stored[c]) else False, "MMA before a CTA stored its scales"
                 for c in (0, 1):
-                    in_flight.append(f"empty{c}.{stage}")
+                    in_flight.append(arrive(f"empty{c}.{stage}"))
                 stage = (stage + 1) % stages
                 sfb = (sfb + 1) % SF_BUFS
                 g += 1
             for c in (0, 1):
-                in_flight.append(f"accf{c}.{a}")
+                in_flight.append(arrive(f"accf{c}.{a}"))
+
+    stored = {c: [] for c in (0, 1)}
 
     def sf_writers(c):
-        full_uses = [0] * stages
+        land_uses = [0] * stages
         released = [0] * stages
         stage, sfb, n = 0, 0, 0
-        for _ in range(n_tiles * slots):
-            yield from wait("sf.full", f"full{c}.{stage}", full_uses[stage])
-            full_uses[stage] += 1
+        for g in range(n_tiles * slots):
+            yield from wait("sf.land", f"sf_land{c}.{stage}", land_uses[stage])
+            land_uses[stage] += 1
+            has_sf = g % slots >= lr_slots
+            if has_sf:
+                assert done(f"sf_land{c}.{stage}") >= land_uses[stage], "scales read before they landed"
             if n >= SF_BUFS:
                 ps = (stage - SF_BUFS) % stages
                 yield from wait("sf.release", f"empty{c}.{ps}", released[ps])
                 released[ps] += 1
+            # the scale buffer this slot writes was last read by the MMAs of slot n - SF_BUFS
+            assert n < SF_BUFS or done(f"empty{c}.{(stage - SF_BUFS) % stages}") >= \
+                (n - SF_BUFS) // stages + 1, "scale buffer rewritten while its MMAs read it"
+            stored[c].append(True)
             B[f"sf_full{sfb}"].arrive(4)
             n += 1
             stage = (stage + 1) % stages
@@ -135,10 +183,10 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
                 raise AssertionError(f"deadlock: {still}")
         rng.shuffle(in_flight)
         for _ in range(rng.randint(0, len(in_flight))):
-            B[in_flight.pop()].arrive()
+            in_flight.pop()()
     assert not live, "model did not finish"
     while in_flight:
-        B[in_flight.pop()].arrive()
+        in_flight.pop()()
     for name, b in B.items():
         assert b.pending == b.count, f"{name}: {b.count - b.pending} stray arrivals at the end"
     return True
