@@ -124,6 +124,31 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   return v;
 }
 
+// Largest magnitude of 16 values, as a balanced tree of 3-input maxima (depth 3 instead of a
+// 16-long running max).
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float r;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float amax16(const float2 (&v)[8]) {
+  const float m0 = max3_abs(v[0].x, v[0].y, v[1].x), m1 = max3_abs(v[1].y, v[2].x, v[2].y);
+  const float m2 = max3_abs(v[3].x, v[3].y, v[4].x), m3 = max3_abs(v[4].y, v[5].x, v[5].y);
+  const float m4 = max3_abs(v[6].x, v[6].y, v[7].x);
+  return fmaxf(max3_abs(m0, m1, m2), max3_abs(m3, m4, v[7].y));
+}
+
+// E4M3 code of a block scale, E4M3_rne_sat(fp32(amax / d6)). The quotient is first taken as
+// fp32(amax * rd6) with rd6 = fp32(1 / d6): that is within 3 units in the last place of the
+// correctly rounded quotient, so both round to the same E4M3 value unless it lies within 4 units
+// of an E4M3 rounding boundary (a midpoint between E4M3 values: fp32 mantissa bits 19..0 equal to
+// 0x80000) or below E4M3's normal range (2^-6); there the exact IEEE division decides.
+__device__ __forceinline__ uint32_t block_scale_code(float amax, float d6, float rd6) {
+  float q = __fmul_rn(amax, rd6);
+  if (q < 0.015625f || (__float_as_uint(q) & 0xFFFFFu) - 0x7FFFCu <= 8u) q = __fdiv_rn(amax, d6);
+  return cvt_e4m3(q);
+}
+
 // ------------------------------------------------------------------------------------------------
 // Kernel 1: smoothing + NVFP4 activation quantization + U = X L1s, one pass over X.
 //
@@ -220,7 +245,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   const float gx = *a.g_x;
   const float alpha = __fmul_rn(gx, *a.g_w);
   float* rs_tab = reinterpret_cast<float*>(smem + L::kTabOff);
-  if (threadIdx.x < 128) rs_tab[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_value(threadIdx.x), gx));
+  // 1 / (dec(s) g_x) per scale code; code 0 (an all-zero block, whose codes are forced to +0) gets 0
+  if (threadIdx.x < 128) rs_tab[threadIdx.x] = threadIdx.x ? __frcp_rn(__fmul_rn(e4m3_value(threadIdx.x), gx)) : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -281,6 +307,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     const int t = ((qw & 7) << 5) + lane;
     const int b = t & 3;
     const float d6 = __fmul_rn(6.0f, gx);
+    const float rd6 = __frcp_rn(d6);
     // this thread's code and scale destinations at step 0; each step moves 32 code bytes along the
     // row and one 512-byte scale atom along K
     uint8_t* code_ptr[2];
@@ -288,8 +315,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int row = m_tile * 128 + (t >> 2) + 64 * i;
-      code_ptr[i] = a.codes + static_cast<size_t>(row) * (K >> 1) + ((kbeg + (b << 4)) >> 1);
-      sf_ptr[i] = a.sf + act_sf_offset(row, (kbeg >> 4) + b, K);
+      code_ptr[i] = a.codes + static_cast<size_t>(row) * (K >> 1) + ((kbeg + (b << 4)) >> 1) + (grp << 5);
+      sf_ptr[i] = a.sf + act_sf_offset(row, (kbeg >> 4) + b, K) + (grp << 9);
     }
     int stage = grp;
     uint32_t phase = 0;
@@ -319,29 +346,28 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       for (int i = 0; i < 2; ++i) {
         const uint32_t wx[8] = {x[i][0].x, x[i][0].y, x[i][0].z, x[i][0].w, x[i][1].x, x[i][1].y, x[i][1].z, x[i][1].w};
         float2 v[8];
-        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[j] = mul2_rn(make_float2(__uint_as_float(wx[j] << 16), __uint_as_float(wx[j] & 0xFFFF0000u)), lam[j]);
+        const uint32_t sc = block_scale_code(amax16(v), d6, rd6);
+        // branch-free: a zero scale multiplies by 0 and its codes are then forced to +0
+        const float r = rs_tab[sc];
+        const float2 r2 = make_float2(r, r);
+        float q[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          v[j] = mul2_rn(make_float2(__uint_as_float(wx[j] << 16), __uint_as_float(wx[j] & 0xFFFF0000u)), lam[j]);
-          amax = fmaxf(amax, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
+          const float2 p = mul2_rn(v[j], r2);
+          q[2 * j] = p.x;
+          q[2 * j + 1] = p.y;
         }
-        const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, d6));
-        uint2 codes = make_uint2(0u, 0u);
-        if (sc != 0) {
-          const float r = rs_tab[sc];
-          const float2 r2 = make_float2(r, r);
-          float q[16];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float2 p = mul2_rn(v[j], r2);
-            q[2 * j] = p.x;
-            q[2 * j + 1] = p.y;
-          }
-          codes.x = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q));
-          codes.y = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q + 8));
-        }
-        *reinterpret_cast<uint2*>(code_ptr[i] + (st << 5)) = codes;
-        sf_ptr[i][static_cast<size_t>(st) << 9] = static_cast<uint8_t>(sc);
+        uint2 codes;
+        codes.x = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q));
+        codes.y = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q + 8));
+        if (sc == 0) codes = make_uint2(0u, 0u);
+        *reinterpret_cast<uint2*>(code_ptr[i]) = codes;
+        *sf_ptr[i] = static_cast<uint8_t>(sc);
+        code_ptr[i] += 64;    // two K steps (this group's next stage) of codes
+        sf_ptr[i] += 1024;    // two 512-byte scale atoms
       }
       stage += 2;
       if (stage >= S) { stage -= S; phase ^= 1u; }
