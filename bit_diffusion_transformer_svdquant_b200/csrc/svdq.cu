@@ -96,13 +96,13 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<128, kStagesTile128>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<128, kStagesTile128>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0, svdq::Nvfp4Act>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::Q1Layout<0>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<16, svdq::Nvfp4Act>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::Q1Layout<16>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<32, svdq::Nvfp4Act>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::Q1Layout<32>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<64, svdq::Nvfp4Act>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::Q1Layout<64>::kSmem));
     // How many CTA pairs of each GEMM instantiation can be resident at once: the persistent grid
     // never asks for more (pairs must sit on two SMs of one GPC, so this can be below sms / 2).
@@ -150,19 +150,19 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
       }
       return SVDQ_OK;
     };
-    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<0>), svdq::Q1Layout<0>::kSmem,
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<0, svdq::Nvfp4Act>), svdq::Q1Layout<0>::kSmem,
                                     st.k1_clusters[0]);
         s != SVDQ_OK)
       return s;
-    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<16>),
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<16, svdq::Nvfp4Act>),
                                     svdq::Q1Layout<16>::kSmem, st.k1_clusters[1]);
         s != SVDQ_OK)
       return s;
-    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<32>),
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<32, svdq::Nvfp4Act>),
                                     svdq::Q1Layout<32>::kSmem, st.k1_clusters[2]);
         s != SVDQ_OK)
       return s;
-    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<64>),
+    if (svdq_status s = k1_clusters(reinterpret_cast<const void*>(svdq::quant_act_kernel<64, svdq::Nvfp4Act>),
                                     svdq::Q1Layout<64>::kSmem, st.k1_clusters[3]);
         s != SVDQ_OK)
       return s;
@@ -541,19 +541,19 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
   switch (r) {
     case 0:
       cfg.dynamicSmemBytes = svdq::Q1Layout<0>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<0>, tmX, tmL1, a);
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<0, svdq::Nvfp4Act>, tmX, tmL1, a);
       break;
     case 16:
       cfg.dynamicSmemBytes = svdq::Q1Layout<16>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<16>, tmX, tmL1, a);
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<16, svdq::Nvfp4Act>, tmX, tmL1, a);
       break;
     case 32:
       cfg.dynamicSmemBytes = svdq::Q1Layout<32>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<32>, tmX, tmL1, a);
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<32, svdq::Nvfp4Act>, tmX, tmL1, a);
       break;
     case 64:
       cfg.dynamicSmemBytes = svdq::Q1Layout<64>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<64>, tmX, tmL1, a);
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<64, svdq::Nvfp4Act>, tmX, tmL1, a);
       break;
     default: return fail(SVDQ_ERR_UNSUPPORTED, "r=%d unsupported", r);
   }
@@ -731,14 +731,14 @@ svdq_status fp8r_ready(int* dev_out, int* sm_out) {
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, L192::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::gemm_kernel<128, kFp8Stages128>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, L128::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<0>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<16>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<32>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::quant_act_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   svdq::QuantLayout<64>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0, svdq::fp8r::RowAct>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::Q1Layout<0>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<16, svdq::fp8r::RowAct>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::Q1Layout<16>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<32, svdq::fp8r::RowAct>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::Q1Layout<32>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<64, svdq::fp8r::RowAct>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::Q1Layout<64>::kSmem));
     if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::fp8r::gemm_kernel<256, kFp8Stages256>),
                                        L256::kSmem, sms, &st.max_pairs[0]);
         s != SVDQ_OK)
@@ -947,11 +947,15 @@ svdq_status svdq_fp8r_quantize_act(const uint16_t* X, const svdq_fp8r_weight* w,
         s != SVDQ_OK)
       return s;
   }
-  // K split over a cluster as for the NVFP4 kernel 1 (same structure and stage sizes)
+  // K split over a cluster exactly as for the NVFP4 kernel 1 (the same kernel body and resources)
   const int m_tiles = act->M_pad / 128;
   int csize = 1;
-  if (m_tiles < 2 * sms && (K / 2) % 64 == 0) csize = 2;
-  if (16 * m_tiles <= sms && (K / 4) % 64 == 0) csize = 4;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    const int* mc = g_dev[dev].k1_clusters[r == 0 ? 0 : r == 16 ? 1 : r == 32 ? 2 : 3];
+    if (m_tiles <= mc[1] && (K / 2) % 64 == 0) csize = 2;
+    if (m_tiles <= mc[2] && (K / 4) % 64 == 0) csize = 4;
+  }
   svdq::fp8r::ActArgs a;
   a.inv_lambda = w->inv_lambda;
   a.rs_x = act->row_rscale;
@@ -970,32 +974,32 @@ svdq_status svdq_fp8r_quantize_act(const uint16_t* X, const svdq_fp8r_weight* w,
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(m_tiles * csize, 1, 1);
-  cfg.blockDim = dim3(svdq::kQThreads, 1, 1);
+  cfg.blockDim = dim3(svdq::kQ1Threads, 1, 1);
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaSuccess;
   switch (r) {
     case 0:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<0>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<0>, tmX, tmL1, a);
+      cfg.dynamicSmemBytes = svdq::Q1Layout<0>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<0, svdq::fp8r::RowAct>, tmX, tmL1, a);
       break;
     case 16:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<16>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<16>, tmX, tmL1, a);
+      cfg.dynamicSmemBytes = svdq::Q1Layout<16>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<16, svdq::fp8r::RowAct>, tmX, tmL1, a);
       break;
     case 32:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<32>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<32>, tmX, tmL1, a);
+      cfg.dynamicSmemBytes = svdq::Q1Layout<32>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<32, svdq::fp8r::RowAct>, tmX, tmL1, a);
       break;
     case 64:
-      cfg.dynamicSmemBytes = svdq::QuantLayout<64>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, svdq::fp8r::quant_act_kernel<64>, tmX, tmL1, a);
+      cfg.dynamicSmemBytes = svdq::Q1Layout<64>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, svdq::quant_act_kernel<64, svdq::fp8r::RowAct>, tmX, tmL1, a);
       break;
     default: return fail(SVDQ_ERR_UNSUPPORTED, "r=%d unsupported", r);
   }
-  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of fp8r::quant_act_kernel failed: %s", cudaGetErrorString(e));
-  return check_launch("fp8r::quant_act_kernel");
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of the row-wise FP8 quant_act_kernel failed: %s", cudaGetErrorString(e));
+  return check_launch("quant_act_kernel (row-wise FP8)");
 }
 
 svdq_status svdq_fp8r_gemm(const svdq_fp8r_act* act, const svdq_fp8r_weight* w, const uint16_t* bias,

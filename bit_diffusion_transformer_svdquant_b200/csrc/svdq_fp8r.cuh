@@ -163,133 +163,28 @@ struct ActArgs {
   int M, K, M_pad, k_per_cta;
 };
 
-// Kernel 1 (row-wise FP8): the NVFP4 kernel 1's structure (TMA ring of 128 x 64 bf16 stages and
-// their inverse smoothing factors, eight quantizer warps and a tcgen05 bf16 MMA reading the same
-// stage, K split over a cluster with a DSMEM reduction of U) with a per-element quantizer: thread t
-// of the 256 owns 16-element block t % 4 of rows t / 4 and t / 4 + 64 of each stage and writes its
-// 16 E4M3 codes as one 16-byte store. U is stored times the row's rs_x.
-template <int R>
-__global__ void __launch_bounds__(kQThreads, 2)
-    quant_act_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL1,
-                     const ActArgs a) {
-  using L = QuantLayout<R>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sbase = smem_addr(smem);
-  const uint32_t bar0 = sbase + L::kBarOff;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kQStages + s); };
-  const uint32_t accf_bar = bar0 + 8u * (2 * kQStages);
-  const uint32_t drain_bar = accf_bar + 8u;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t csize = cluster_nctarank(), crank = cluster_ctarank();
-  const int m_tile = blockIdx.x / csize;
-  const int kbeg = static_cast<int>(crank) * a.k_per_cta;
-  const int n_steps = a.k_per_cta >> 6;
-  const int K = a.K;
-  unsigned* status = &g_svdq_status;
-  const uint64_t wait_ns = a.wait_ns;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 8 + (R > 0 ? 1 : 0));
-    }
-    mbar_init(accf_bar, 1);
-    mbar_init(drain_bar, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-    prefetch_tmap(&tmX);
-    if (R > 0) prefetch_tmap(&tmL1);
-  }
-  if (R > 0 && warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = R > 0 ? *tmem_slot : 0u;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, armed = 0, armed_parity = 0;
-      for (int st = 0; st < n_steps; ++st) {
-        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)) break;
-        const uint32_t sa = sbase + stage * L::kStage;
-        mbar_arrive_expect_tx(full_bar(stage), kQTile + R * 128 + 256);
-        const int kx = kbeg + (st << 6);
-        tma_load_2d(sa, &tmX, kx, m_tile * 128, full_bar(stage));
-        if (R > 0) tma_load_2d(sa + kQTile, &tmL1, kx, 0, full_bar(stage));
-        bulk_load(sa + L::kLamOff, a.inv_lambda + kx, 256, full_bar(stage));
-        armed |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kQStages) { stage = 0; phase ^= 1u; }
-      }
-      for (int s = 0; s < kQStages; ++s)
-        if (armed & (1u << s))
-          mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
-    }
-  } else if (warp == 1) {
-    if (R > 0 && lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, accumulate = 0;
-      bool ok = true;
-      const uint32_t idesc = idesc_bf16(128, R);
-      for (int st = 0; st < n_steps; ++st) {
-        if (!(ok = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusMma, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t sa = sbase + stage * L::kStage;
-        const uint64_t dx = smem_desc(sa, 16, 1024, 2);
-        const uint64_t dl = smem_desc(sa + kQTile, 16, 1024, 2);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          mma_bf16(tmem, dx + 2u * j, dl + 2u * j, idesc, accumulate);
-          accumulate = 1;
-        }
-        tc_commit(empty_bar(stage));
-        if (++stage == kQStages) { stage = 0; phase ^= 1u; }
-      }
-      if (ok) tc_commit(accf_bar);
-      tc_commit(drain_bar);
-      mbar_wait_bounded(drain_bar, 0, wait_ns, status, kStatusDrain, nullptr);
-    }
-  } else {
-    const int t = threadIdx.x - 64;
-    const int b = t & 3;
-    // the reciprocal row scales of this thread's two rows (M_pad entries; pad rows hold 1)
-    const float rs0 = a.rs_x[m_tile * 128 + (t >> 2)];
-    const float rs1 = a.rs_x[m_tile * 128 + (t >> 2) + 64];
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int st = 0; st < n_steps; ++st) {
-      const bool got = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;
-      const int k = kbeg + (st << 6) + (b << 4);
-      const uint8_t* tile = smem + stage * L::kStage;
-      float2 lam[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 l = reinterpret_cast<const float4*>(tile + L::kLamOff)[4 * b + j];
-        lam[2 * j] = make_float2(l.x, l.y);
-        lam[2 * j + 1] = make_float2(l.z, l.w);
-      }
-      uint4 x[2][2];
+// Kernel 1 (row-wise FP8) is svdq::quant_act_kernel with this quantizer policy: each thread
+// turns its two 16-element blocks of a stage into E4M3 codes q = E4M3_sat(fp32(x_hat * rs_x))
+// with its rows' reciprocal scales (written by act_row_scale_kernel before the launch) and stores
+// each block's 16 codes as one 16-byte store; U is stored times the row's rs_x.
+struct RowAct {
+  using Args = ActArgs;
+  __device__ static void prologue(const Args&, float*) {}
+  struct Thread {
+    float rs[2];
+    uint8_t* code_ptr[2];
+    __device__ Thread(const Args& a, const float*, int m_tile, int rl, int b, int kbeg, int grp) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int rl = (t >> 2) + 64 * i;
-        x[i][0] = *reinterpret_cast<const uint4*>(tile + rl * 128 + (((2 * b) ^ (rl & 7)) << 4));
-        x[i][1] = *reinterpret_cast<const uint4*>(tile + rl * 128 + (((2 * b + 1) ^ (rl & 7)) << 4));
+        const int row = m_tile * 128 + rl + 64 * i;
+        rs[i] = a.rs_x[row];  // M_pad entries; pad rows hold 1
+        code_ptr[i] = a.codes + static_cast<size_t>(row) * a.K + kbeg + (b << 4) + (grp << 6);
       }
+    }
+    __device__ void stage(const float2 (&lam)[8], const uint4 (&x)[2][2]) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int rl = (t >> 2) + 64 * i;
-        const float rs = i == 0 ? rs0 : rs1;
-        const float2 r2 = make_float2(rs, rs);
+        const float2 r2 = make_float2(rs[i], rs[i]);
         const uint32_t wx[8] = {x[i][0].x, x[i][0].y, x[i][0].z, x[i][0].w, x[i][1].x, x[i][1].y, x[i][1].z, x[i][1].w};
         uint32_t w[4];
 #pragma unroll
@@ -300,93 +195,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
           const float2 q0 = mul2_rn(v0, r2), q1 = mul2_rn(v1, r2);
           w[j >> 1] = cvt_e4m3x2(q0.x, q0.y) | (cvt_e4m3x2(q1.x, q1.y) << 16);
         }
-        const int row = m_tile * 128 + rl;
-        *reinterpret_cast<uint4*>(a.codes + static_cast<size_t>(row) * K + k) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar(stage));
-      if (++stage == kQStages) { stage = 0; phase ^= 1u; }
-    }
-    if constexpr (R > 0) {
-      // warps 2..5 (quadrant q = warp % 4) read this CTA's rows of U from TMEM; cluster members
-      // park their partials in shared memory and the cluster's first CTA adds them in rank order
-      const int q = warp & 3;
-      const bool mine_rows = warp < 6;
-      bool got = true;
-      if (mine_rows) got = mbar_wait_bounded(accf_bar, 0, wait_ns, status, kStatusEpilogue, abort_flag);
-      got = __all_sync(0xffffffffu, got) && mine_rows;
-      float u[R];
-#pragma unroll
-      for (int j = 0; j < R; ++j) u[j] = 0.0f;
-      if (got) {
-        tc_fence_after();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16);
-        if constexpr (R == 16) {
-          float t16[16];
-          tmem_ld_32x16(ta, t16);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) u[e] = t16[e];
-        } else {
-#pragma unroll
-          for (int j = 0; j < R; j += 32) {
-            float t32[32];
-            tmem_ld_32x32(ta + j, t32);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[j + e] = t32[e];
-          }
-        }
-        if (csize > 1 && crank != 0) {
-          float* part = reinterpret_cast<float*>(smem + L::kPartOff) + (q * 32 + lane) * (R + 1);
-#pragma unroll
-          for (int j = 0; j < R; ++j) part[j] = u[j];
-        }
-      }
-      if (csize > 1) cluster_sync_all();
-      if (got && crank == 0) {
-        const int rl = q * 32 + lane;
-        for (uint32_t rk = 1; rk < csize; ++rk) {
-          const uint32_t pa = cluster_map(smem_addr(smem + L::kPartOff) + rl * (R + 1) * 4, rk);
-#pragma unroll
-          for (int j = 0; j < R; ++j) u[j] += ld_cluster_f32(pa + j * 4);
-        }
-        const float cinv = a.rs_x[m_tile * 128 + rl];
-        __nv_bfloat16* u_hi = a.U + (static_cast<size_t>(m_tile) * 128 + rl) * R;
-        __nv_bfloat16* u_lo = u_hi + static_cast<size_t>(a.M_pad) * R;
-#pragma unroll
-        for (int j = 0; j < R; j += 8) {
-          uint32_t wh[4], wl[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float v0 = __fmul_rn(u[j + 2 * e], cinv), v1 = __fmul_rn(u[j + 2 * e + 1], cinv);
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(v0, v1);
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(__fsub_rn(v0, __low2float(hi)), __fsub_rn(v1, __high2float(hi)));
-            wh[e] = *reinterpret_cast<const uint32_t*>(&hi);
-            wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
-          }
-          *reinterpret_cast<uint4*>(u_hi + j) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          *reinterpret_cast<uint4*>(u_lo + j) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-        }
+        *reinterpret_cast<uint4*>(code_ptr[i]) = make_uint4(w[0], w[1], w[2], w[3]);
+        code_ptr[i] += 128;  // two K steps: this group's next stage
       }
     }
-  }
-
-  if constexpr (R == 0) {
-    if (csize > 1) cluster_sync_all();
-  } else {
-    // warps 0 and 1 take part in the cluster barrier the quantizer warps passed above
-    if (csize > 1 && warp < 2) cluster_sync_all();
-  }
-  // peers keep their shared memory until the leader has read it
-  if (csize > 1) cluster_sync_all();
-  tc_fence_before();
-  __syncthreads();
-  if (R > 0 && warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, L::kTmemCols);
-  }
-}
+  };
+  __device__ static float u_scale(const Args& a, int row) { return a.rs_x[row]; }
+  __device__ static void finish(const Args&) {}
+};
 
 // ------------------------------------------------------------------------------------------------
 // Kernel 2 (row-wise FP8): CTA-pair tcgen05 GEMM, kind::f8f6f4.

@@ -138,19 +138,20 @@ __device__ __forceinline__ float amax16(const float2 (&v)[8]) {
   return fmaxf(max3_abs(m0, m1, m2), max3_abs(m3, m4, v[7].y));
 }
 
-// E4M3 code of a block scale, E4M3_rne_sat(fp32(amax / d6)). The quotient is first taken as
-// fp32(amax * rd6) with rd6 = fp32(1 / d6): that is within 3 units in the last place of the
-// correctly rounded quotient, so both round to the same E4M3 value unless it lies within 4 units
-// of an E4M3 rounding boundary (a midpoint between E4M3 values: fp32 mantissa bits 19..0 equal to
-// 0x80000) or below E4M3's normal range (2^-6); there the exact IEEE division decides.
-__device__ __forceinline__ uint32_t block_scale_code(float amax, float d6, float rd6) {
-  float q = __fmul_rn(amax, rd6);
-  if (q < 0.015625f || (__float_as_uint(q) & 0xFFFFFu) - 0x7FFFCu <= 8u) q = __fdiv_rn(amax, d6);
-  return cvt_e4m3(q);
+// The E4M3 code of a block scale is E4M3_rne_sat(fp32(amax / d6)). Kernel 1 first takes the
+// quotient as q = fp32(amax * rd6) with rd6 = fp32(1 / d6): q is within 3 units in the last place
+// of the correctly rounded quotient, so both round to the same E4M3 value unless q lies within 4
+// units of an E4M3 rounding boundary (a midpoint between E4M3 values: fp32 mantissa bits 19..0
+// equal to 0x80000) or below E4M3's normal range (2^-6). This tells whether the exact IEEE
+// division must decide.
+__device__ __forceinline__ bool scale_needs_division(float q) {
+  return q < 0.015625f || (__float_as_uint(q) & 0xFFFFFu) - 0x7FFFCu <= 8u;
 }
 
 // ------------------------------------------------------------------------------------------------
-// Kernel 1: smoothing + NVFP4 activation quantization + U = X L1s, one pass over X.
+// Kernel 1: smoothing + activation quantization + U = X L1s, one pass over X. One kernel body
+// serves both formats; a policy class supplies the quantizer (Nvfp4Act here, the row-wise FP8
+// RowAct in svdq_fp8r.cuh) and the scale U is stored with.
 //
 // A CTA (one per SM) owns 128 rows of X and a K range: the whole K, or a share of it when a
 // thread-block cluster of 2 or 4 CTAs splits K so that few row tiles still fill the SMs in one
@@ -197,10 +198,99 @@ struct QuantActArgs {
   int M, K, M_pad, k_per_cta;
 };
 
-template <int R>
+// The NVFP4 quantizer of kernel 1 (a policy of quant_act_kernel). Rounding points as in the
+// header of this file; the per-scale-code reciprocals 1 / (dec(s) g_x) live in a 128-entry table
+// in shared memory (entry 0, an all-zero block whose codes are forced to +0, holds 0).
+struct Nvfp4Act {
+  using Args = QuantActArgs;
+  __device__ static void prologue(const Args& a, float* tab) {
+    const float gx = *a.g_x;
+    if (threadIdx.x < 128) tab[threadIdx.x] = threadIdx.x ? __frcp_rn(__fmul_rn(e4m3_value(threadIdx.x), gx)) : 0.0f;
+  }
+  // One quantizer thread: 16-element block b of local rows rl and rl + 64 of every stage its
+  // group takes (every other stage from `grp` on).
+  struct Thread {
+    float d6, rd6;
+    const float* tab;
+    uint8_t* code_ptr[2];
+    uint8_t* sf_ptr[2];
+    __device__ Thread(const Args& a, const float* tab_, int m_tile, int rl, int b, int kbeg, int grp) : tab(tab_) {
+      d6 = __fmul_rn(6.0f, *a.g_x);
+      rd6 = __frcp_rn(d6);
+      // code and scale destinations at the group's first stage; a group step moves 64 code bytes
+      // along the row and two 512-byte scale atoms along K
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int row = m_tile * 128 + rl + 64 * i;
+        code_ptr[i] = a.codes + static_cast<size_t>(row) * (a.K >> 1) + ((kbeg + (b << 4)) >> 1) + (grp << 5);
+        sf_ptr[i] = a.sf + act_sf_offset(row, (kbeg >> 4) + b, a.K) + (grp << 9);
+      }
+    }
+    // the two blocks go through each phase together, so that their dependency chains interleave
+    __device__ void stage(const float2 (&lam)[8], const uint4 (&x)[2][2]) {
+      float2 v[2][8];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t wx[8] = {x[i][0].x, x[i][0].y, x[i][0].z, x[i][0].w, x[i][1].x, x[i][1].y, x[i][1].z, x[i][1].w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[i][j] = mul2_rn(make_float2(__uint_as_float(wx[j] << 16), __uint_as_float(wx[j] & 0xFFFF0000u)), lam[j]);
+      }
+      float am[2], qs[2];
+      bool exact = false;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        am[i] = amax16(v[i]);
+        qs[i] = __fmul_rn(am[i], rd6);
+        exact |= scale_needs_division(qs[i]);
+      }
+      if (exact) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          if (scale_needs_division(qs[i])) qs[i] = __fdiv_rn(am[i], d6);
+      }
+      uint32_t sc[2];
+      float rr[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        sc[i] = cvt_e4m3(qs[i]);
+        rr[i] = tab[sc[i]];  // a zero scale multiplies by 0 and its codes are then forced to +0
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float2 r2 = make_float2(rr[i], rr[i]);
+        float q[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 p = mul2_rn(v[i][j], r2);
+          q[2 * j] = p.x;
+          q[2 * j + 1] = p.y;
+        }
+        uint2 codes;
+        codes.x = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q));
+        codes.y = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q + 8));
+        if (sc[i] == 0) codes = make_uint2(0u, 0u);
+        *reinterpret_cast<uint2*>(code_ptr[i]) = codes;
+        *sf_ptr[i] = static_cast<uint8_t>(sc[i]);
+        code_ptr[i] += 64;
+        sf_ptr[i] += 1024;
+      }
+    }
+  };
+  // U is stored divided by alpha = fp32(g_x g_w): one scale for the whole GEMM
+  __device__ static float u_scale(const Args& a, int row) {
+    (void)row;
+    return __frcp_rn(__fmul_rn(*a.g_x, *a.g_w));
+  }
+  __device__ static void finish(const Args& a) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *a.alpha = __fmul_rn(*a.g_x, *a.g_w);
+  }
+};
+
+template <int R, class Q>
 __global__ void __launch_bounds__(kQ1Threads, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL1,
-                     const QuantActArgs a) {
+                     const typename Q::Args a) {
   using L = Q1Layout<R>;
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -242,11 +332,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const float gx = *a.g_x;
-  const float alpha = __fmul_rn(gx, *a.g_w);
-  float* rs_tab = reinterpret_cast<float*>(smem + L::kTabOff);
-  // 1 / (dec(s) g_x) per scale code; code 0 (an all-zero block, whose codes are forced to +0) gets 0
-  if (threadIdx.x < 128) rs_tab[threadIdx.x] = threadIdx.x ? __frcp_rn(__fmul_rn(e4m3_value(threadIdx.x), gx)) : 0.0f;
+  float* tab = reinterpret_cast<float*>(smem + L::kTabOff);
+  Q::prologue(a, tab);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -306,18 +393,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     const int grp = qw >> 3;
     const int t = ((qw & 7) << 5) + lane;
     const int b = t & 3;
-    const float d6 = __fmul_rn(6.0f, gx);
-    const float rd6 = __frcp_rn(d6);
-    // this thread's code and scale destinations at step 0; each step moves 32 code bytes along the
-    // row and one 512-byte scale atom along K
-    uint8_t* code_ptr[2];
-    uint8_t* sf_ptr[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int row = m_tile * 128 + (t >> 2) + 64 * i;
-      code_ptr[i] = a.codes + static_cast<size_t>(row) * (K >> 1) + ((kbeg + (b << 4)) >> 1) + (grp << 5);
-      sf_ptr[i] = a.sf + act_sf_offset(row, (kbeg >> 4) + b, K) + (grp << 9);
-    }
+    typename Q::Thread qt(a, tab, m_tile, t >> 2, b, kbeg, grp);
     int stage = grp;
     uint32_t phase = 0;
     for (int st = grp; st < n_steps; st += 2) {
@@ -342,33 +418,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(stage));  // the stage's data is in registers
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint32_t wx[8] = {x[i][0].x, x[i][0].y, x[i][0].z, x[i][0].w, x[i][1].x, x[i][1].y, x[i][1].z, x[i][1].w};
-        float2 v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          v[j] = mul2_rn(make_float2(__uint_as_float(wx[j] << 16), __uint_as_float(wx[j] & 0xFFFF0000u)), lam[j]);
-        const uint32_t sc = block_scale_code(amax16(v), d6, rd6);
-        // branch-free: a zero scale multiplies by 0 and its codes are then forced to +0
-        const float r = rs_tab[sc];
-        const float2 r2 = make_float2(r, r);
-        float q[16];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float2 p = mul2_rn(v[j], r2);
-          q[2 * j] = p.x;
-          q[2 * j + 1] = p.y;
-        }
-        uint2 codes;
-        codes.x = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q));
-        codes.y = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q + 8));
-        if (sc == 0) codes = make_uint2(0u, 0u);
-        *reinterpret_cast<uint2*>(code_ptr[i]) = codes;
-        *sf_ptr[i] = static_cast<uint8_t>(sc);
-        code_ptr[i] += 64;    // two K steps (this group's next stage) of codes
-        sf_ptr[i] += 1024;    // two 512-byte scale atoms
-      }
+      qt.stage(lam, x);
       stage += 2;
       if (stage >= S) { stage -= S; phase ^= 1u; }
     }
@@ -422,7 +472,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
 #pragma unroll
           for (int j = 0; j < R; ++j) u[j] += ld_cluster_f32(pa + j * 4);
         }
-        const float cinv = __frcp_rn(alpha);
+        const float cinv = Q::u_scale(a, m_tile * 128 + rl);
         __nv_bfloat16* u_hi = a.U + (static_cast<size_t>(m_tile) * 128 + rl) * R;
         __nv_bfloat16* u_lo = u_hi + static_cast<size_t>(a.M_pad) * R;
 #pragma unroll
@@ -449,7 +499,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     // warps 0 and 1 take part in the cluster barrier the quantizer warps passed above
     if (csize > 1 && warp < 2) cluster_sync_all();
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.alpha = alpha;
+  Q::finish(a);
   // peers keep their shared memory until the leader has read it
   if (csize > 1) cluster_sync_all();
   tc_fence_before();
@@ -459,26 +509,6 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     tmem_dealloc(tmem, L::kTmemCols);
   }
 }
-
-// The ring layout of kernel 1 as it was before the two-group rewrite, still used by the row-wise
-// FP8 variant's quantizing kernel (four stages, eight quantizer warps, two CTAs per SM).
-constexpr int kQThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 quantize (2..5 also drain U)
-constexpr int kQStages = 4;
-
-template <int R>
-struct QuantLayout {
-  static constexpr int kL1 = (R * 128 + 1023) / 1024 * 1024;
-  static constexpr int kLamOff = kQTile + kL1;
-  static constexpr int kStage = kQTile + kL1 + 1024;
-  static constexpr int kPartOff = kQStages * kStage;
-  static constexpr int kPart = R * 128 * 4 + 128 * 4;
-  static constexpr int kTabOff = kPartOff + kPart;
-  static constexpr int kBarOff = kTabOff + 128 * 4;
-  static constexpr int kNumBars = 2 * kQStages + 2;
-  static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
-  static constexpr int kTmemCols = R <= 32 ? 32 : 64;
-  static_assert(kStage % 1024 == 0, "stage alignment");
-};
 
 // ------------------------------------------------------------------------------------------------
 // Offline pack and calibration helpers.
