@@ -87,13 +87,13 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
         return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
       g_encode = reinterpret_cast<Encode>(fn);
     }
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<256, kStagesTile256>,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 256, kStagesTile256>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<256, kStagesTile256>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<192, kStagesTile192>,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 192, kStagesTile192>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<192, kStagesTile192>::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::svdq_gemm_kernel<128, kStagesTile128>,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 128, kStagesTile128>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<128, kStagesTile128>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0, svdq::Nvfp4Act>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -117,15 +117,15 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
       *out = n;
       return SVDQ_OK;
     };
-    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::svdq_gemm_kernel<256, kStagesTile256>),
+    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 256, kStagesTile256>),
                                   svdq::GemmLayout<256, kStagesTile256>::kSmem, &st.max_pairs[0]);
         s != SVDQ_OK)
       return s;
-    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::svdq_gemm_kernel<192, kStagesTile192>),
+    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 192, kStagesTile192>),
                                   svdq::GemmLayout<192, kStagesTile192>::kSmem, &st.max_pairs[1]);
         s != SVDQ_OK)
       return s;
-    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::svdq_gemm_kernel<128, kStagesTile128>),
+    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 128, kStagesTile128>),
                                   svdq::GemmLayout<128, kStagesTile128>::kSmem, &st.max_pairs[2]);
         s != SVDQ_OK)
       return s;
@@ -631,16 +631,16 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
   const dim3 grid(2 * pairs);  // clusters of 2 CTAs (compiled into the kernel)
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (n_tile == 256) {
-    svdq::svdq_gemm_kernel<256, kStagesTile256><<<grid, svdq::kGemmThreads, svdq::GemmLayout<256, kStagesTile256>::kSmem, st>>>(
+    svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 256, kStagesTile256><<<grid, svdq::kGemmThreads, svdq::GemmLayout<256, kStagesTile256>::kSmem, st>>>(
         tmA, tmB, tmU, tmL2, tmY, g);
   } else if (n_tile == 192) {
-    svdq::svdq_gemm_kernel<192, kStagesTile192><<<grid, svdq::kGemmThreads, svdq::GemmLayout<192, kStagesTile192>::kSmem, st>>>(
+    svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 192, kStagesTile192><<<grid, svdq::kGemmThreads, svdq::GemmLayout<192, kStagesTile192>::kSmem, st>>>(
         tmA, tmB, tmU, tmL2, tmY, g);
   } else {
-    svdq::svdq_gemm_kernel<128, kStagesTile128><<<grid, svdq::kGemmThreads, svdq::GemmLayout<128, kStagesTile128>::kSmem, st>>>(
+    svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 128, kStagesTile128><<<grid, svdq::kGemmThreads, svdq::GemmLayout<128, kStagesTile128>::kSmem, st>>>(
         tmA, tmB, tmU, tmL2, tmY, g);
   }
-  return check_launch("svdq_gemm_kernel");
+  return check_launch("pair_gemm_kernel (NVFP4)");
 }
 
 svdq_status svdq_export_weight(const svdq_weight* w, uint8_t* codes, uint8_t* scales, svdq_stream_t stream) {
@@ -722,14 +722,14 @@ svdq_status fp8r_ready(int* dev_out, int* sm_out) {
   std::lock_guard<std::mutex> lk(g_dev_mu);
   Fp8rState& st = g_fp8r[dev];
   if (!st.ready) {
-    using L256 = svdq::fp8r::GemmLayout<256, kFp8Stages256>;
-    using L192 = svdq::fp8r::GemmLayout<192, kFp8Stages192>;
-    using L128 = svdq::fp8r::GemmLayout<128, kFp8Stages128>;
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::gemm_kernel<256, kFp8Stages256>,
+    using L256 = svdq::PairGemmLayout<false, 256, kFp8Stages256>;
+    using L192 = svdq::PairGemmLayout<false, 192, kFp8Stages192>;
+    using L128 = svdq::PairGemmLayout<false, 128, kFp8Stages128>;
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 256, kFp8Stages256>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, L256::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::gemm_kernel<192, kFp8Stages192>,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 192, kFp8Stages192>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, L192::kSmem));
-    SVDQ_CUDA(cudaFuncSetAttribute(svdq::fp8r::gemm_kernel<128, kFp8Stages128>,
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 128, kFp8Stages128>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, L128::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0, svdq::fp8r::RowAct>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::Q1Layout<0>::kSmem));
@@ -739,15 +739,15 @@ svdq_status fp8r_ready(int* dev_out, int* sm_out) {
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::Q1Layout<32>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<64, svdq::fp8r::RowAct>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::Q1Layout<64>::kSmem));
-    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::fp8r::gemm_kernel<256, kFp8Stages256>),
+    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 256, kFp8Stages256>),
                                        L256::kSmem, sms, &st.max_pairs[0]);
         s != SVDQ_OK)
       return s;
-    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::fp8r::gemm_kernel<192, kFp8Stages192>),
+    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 192, kFp8Stages192>),
                                        L192::kSmem, sms, &st.max_pairs[1]);
         s != SVDQ_OK)
       return s;
-    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::fp8r::gemm_kernel<128, kFp8Stages128>),
+    if (svdq_status s = fp8r_max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 128, kFp8Stages128>),
                                        L128::kSmem, sms, &st.max_pairs[2]);
         s != SVDQ_OK)
       return s;
@@ -1071,16 +1071,16 @@ svdq_status svdq_fp8r_gemm(const svdq_fp8r_act* act, const svdq_fp8r_weight* w, 
   const dim3 grid(2 * pairs);  // clusters of 2 CTAs (compiled into the kernel)
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (n_tile == 256) {
-    svdq::fp8r::gemm_kernel<256, kFp8Stages256>
-        <<<grid, svdq::kGemmThreads, svdq::fp8r::GemmLayout<256, kFp8Stages256>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
+    svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 256, kFp8Stages256>
+        <<<grid, svdq::kGemmThreads, svdq::PairGemmLayout<false, 256, kFp8Stages256>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
   } else if (n_tile == 192) {
-    svdq::fp8r::gemm_kernel<192, kFp8Stages192>
-        <<<grid, svdq::kGemmThreads, svdq::fp8r::GemmLayout<192, kFp8Stages192>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
+    svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 192, kFp8Stages192>
+        <<<grid, svdq::kGemmThreads, svdq::PairGemmLayout<false, 192, kFp8Stages192>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
   } else {
-    svdq::fp8r::gemm_kernel<128, kFp8Stages128>
-        <<<grid, svdq::kGemmThreads, svdq::fp8r::GemmLayout<128, kFp8Stages128>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
+    svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 128, kFp8Stages128>
+        <<<grid, svdq::kGemmThreads, svdq::PairGemmLayout<false, 128, kFp8Stages128>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
   }
-  return check_launch("fp8r::gemm_kernel");
+  return check_launch("pair_gemm_kernel (row-wise FP8)");
 }
 
 svdq_status svdq_fp8r_export_weight(const svdq_fp8r_weight* w, uint8_t* codes, float* scales, svdq_stream_t stream) {

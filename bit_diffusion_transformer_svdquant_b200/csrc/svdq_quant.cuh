@@ -313,6 +313,9 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   unsigned* status = &g_svdq_status;
   const uint64_t wait_ns = a.wait_ns;
 
+  // the first ring fill (one load per slot) is issued by the producer thread right after the barrier
+  // set-up, so its latency overlaps the TMEM allocation and the table set-up of the other warps
+  const int n_pre = n_steps < S ? n_steps : S;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), 1);
@@ -322,8 +325,16 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tmX);
-    if (R > 0) prefetch_tmap(&tmL1);
+    fence_proxy_async_smem();
+    const uint64_t pol_x = l2_policy_evict_first();
+    for (int st = 0; st < n_pre; ++st) {
+      const uint32_t sa = sbase + st * L::kStage;
+      mbar_arrive_expect_tx(full_bar(st), kQTile + R * 128 + 256);
+      const int kx = kbeg + (st << 6);
+      tma_load_2d_hint(sa, &tmX, kx, m_tile * 128, full_bar(st), pol_x);
+      if (R > 0) tma_load_2d(sa + kQTile, &tmL1, kx, 0, full_bar(st));
+      bulk_load(sa + L::kLamOff, a.inv_lambda + kx, 256, full_bar(st));
+    }
   }
   if (R > 0 && warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
@@ -342,9 +353,11 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   if (warp == 0) {
     if (lane == 0) {
       const uint64_t pol_x = l2_policy_evict_first();
-      int stage = 0;
-      uint32_t phase = 0, armed = 0, armed_parity = 0;
-      for (int st = 0; st < n_steps; ++st) {
+      // stages 0 .. n_pre - 1 went out with the set-up (phase 0 of their slots)
+      int stage = n_pre == S ? 0 : n_pre;
+      uint32_t phase = n_pre == S ? 1u : 0u;
+      uint32_t armed = (1u << n_pre) - 1u, armed_parity = 0;
+      for (int st = n_pre; st < n_steps; ++st) {
         if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)) break;
         const uint32_t sa = sbase + stage * L::kStage;
         mbar_arrive_expect_tx(full_bar(stage), kQTile + R * 128 + 256);

@@ -1,7 +1,8 @@
-"""A discrete-event model of the barrier protocol of the NVFP4 CTA-pair GEMM (svdq_gemm_kernel in
-csrc/svdq_gemm.cuh), checked on the host like test_fused_protocol_model.py: producer, MMA issuer,
-the four scale-factor writer warps and the eight epilogue warps of both CTAs replay their barrier
-traffic in the kernel's order, with copies and MMA completions landing late and in random order.
+"""A discrete-event model of the barrier protocol of the CTA-pair GEMM (pair_gemm_kernel in
+csrc/svdq_gemm.cuh, for both formats: NVFP4 with its scale factors, and row-wise FP8 without),
+checked on the host like test_fused_protocol_model.py: producer, MMA issuer, the four scale-factor
+writer warps (NVFP4 only) and the eight epilogue warps of both CTAs replay their barrier traffic in
+the kernel's order, with copies and MMA completions landing late and in random order.
 
 Protocol per ring slot: both CTAs' A / B (or low-rank) copies complete on the even CTA's full
 barrier, whose phase also needs the even producer's arrive (it expects both CTAs' bytes); each CTA's
@@ -11,10 +12,11 @@ the issuer waits for full and sf_full, issues the MMAs and commits to both CTAs'
 At the end each producer waits for the release of every slot it filled, so no copy is in flight
 when its CTA exits.
 
-Both accumulator modes are covered: one 256- or 192-column buffer (5-stage ring), and two
-128-column buffers used alternately (6-stage ring). Checked: no deadlock, no stray arrival, waits on
-exactly their completion, no resource used before its previous user is done; removing any one wait
-must make it fail."""
+Both accumulator modes are covered: one 256- or 192-column buffer (NVFP4, 5-stage ring), and two
+buffers used alternately (NVFP4 128-wide tiles with a 6-stage ring, and every FP8 tile width with
+6- and 8-stage rings, where without scale factors the issuer waits on the full barrier alone).
+Checked: no deadlock, no stray arrival, waits on exactly their completion, no resource used before
+its previous user is done; removing any one wait must make it fail."""
 import random
 
 import pytest
@@ -36,7 +38,7 @@ class Barrier:
             self.pending = self.count
 
 
-def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
+def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=(), scales=True):
     rng = random.Random(seed)
     lr_slots = (r + 31) // 32
     slots = lr_slots + k_iters
@@ -87,11 +89,12 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
             yield from wait("producer.empty", f"empty{c}.{stage}", uses[stage] - 1)
             assert done(f"empty{c}.{stage}") >= uses[stage], "ring stage refilled while its MMAs read it"
             uses[stage] += 1
-            if has_sf:
-                B[f"sf_land{c}.{stage}"].arrive()
-                in_flight.append(arrive(f"sf_land{c}.{stage}"))
-            else:
-                B[f"sf_land{c}.{stage}"].arrive(2)
+            if scales:
+                if has_sf:
+                    B[f"sf_land{c}.{stage}"].arrive()
+                    in_flight.append(arrive(f"sf_land{c}.{stage}"))
+                else:
+                    B[f"sf_land{c}.{stage}"].arrive(2)
             if c == 0:
                 B[f"full.{stage}"].arrive()
             issued[c][stage] += 1
@@ -111,11 +114,13 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
             assert done(f"acce{a}") >= use, "accumulator overwritten before its epilogue read it"
             for _ in range(slots):
                 yield from wait("issuer.full", f"full.{stage}", g // stages)
-                yield from wait("issuer.sf_full", f"sf_full{sfb}", sf_uses[sfb])
-                sf_uses[sfb] += 1
+                if scales:
+                    yield from wait("issuer.sf_full", f"sf_full{sfb}", sf_uses[sfb])
+                    sf_uses[sfb] += 1
                 for c in (0, 1):
                     assert landed[c][stage] >= g // stages + 1, "MMA before a CTA's copy landed"
-                    assert stored[c][g] if g < len(stored[c]) else False, "MMA before a CTA stored its scales"
+                    if scales:
+                        assert stored[c][g] if g < len(stored[c]) else False, "MMA before a CTA stored its scales"
                 for c in (0, 1):
                     in_flight.append(arrive(f"empty{c}.{stage}"))
                 stage = (stage + 1) % stages
@@ -159,7 +164,8 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
     live = {"issuer": issuer()}
     for c in (0, 1):
         live[f"producer{c}"] = producer(c)
-        live[f"sf{c}"] = sf_writers(c)
+        if scales:
+            live[f"sf{c}"] = sf_writers(c)
         for w in range(8):
             live[f"epi{c}.{w}"] = epilogue(c)
 
@@ -192,23 +198,29 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=()):
     return True
 
 
-# (stages, accumulator buffers) of the kernel's instantiations: 256 and 192 -> (5, 1), 128 -> (6, 2)
-@pytest.mark.parametrize("stages,acc_bufs", [(5, 1), (6, 2)])
+# (stages, accumulator buffers, scale factors) of the kernel's instantiations: NVFP4 256 / 192 ->
+# (5, 1), NVFP4 128 -> (6, 2); row-wise FP8 256 / 192 -> (6, 2, no scales), 128 -> (8, 2, no scales)
+MODES = [(5, 1, True), (6, 2, True), (6, 2, False), (8, 2, False)]
+
+
+@pytest.mark.parametrize("stages,acc_bufs,scales", MODES)
 @pytest.mark.parametrize("n_tiles", [1, 2, 3, 8])
 @pytest.mark.parametrize("r,k_iters", [(32, 1), (64, 2), (0, 3), (16, 12)])
-def test_nvfp4_protocol_model(stages, acc_bufs, n_tiles, r, k_iters):
+def test_pair_gemm_protocol_model(stages, acc_bufs, scales, n_tiles, r, k_iters):
     for seed in range(5):
-        assert run_model(n_tiles, r, k_iters, stages, acc_bufs, seed)
+        assert run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, scales=scales)
 
 
 @pytest.mark.parametrize("skipped", WAITS)
-@pytest.mark.parametrize("stages,acc_bufs", [(5, 1), (6, 2)])
-def test_every_wait_is_needed(skipped, stages, acc_bufs):
+@pytest.mark.parametrize("stages,acc_bufs,scales", MODES)
+def test_every_wait_is_needed(skipped, stages, acc_bufs, scales):
+    if not scales and skipped.startswith(("sf.", "issuer.sf_")):
+        pytest.skip("no scale factors in this format")
     for n_tiles in (3, 8):
         for r, k_iters in ((32, 1), (0, 3), (16, 12)):
             for seed in range(20):
                 try:
-                    run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip={skipped})
+                    run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip={skipped}, scales=scales)
                 except AssertionError:
                     return
     pytest.fail(f"removing the wait {skipped} went unnoticed")
