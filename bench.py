@@ -40,11 +40,11 @@ FP4_PER_BF16 = 4.0   # nominal dense FP4 / dense bf16 tensor throughput on B200 
 FP8_PER_BF16 = 2.0   # nominal dense FP8 / dense bf16 (4.5 / 2.25 PFLOP/s)
 FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch of the GEMM, from the ncu capture summarised in
-# profiles/svdq_gemm_kernel_qkv2048.md, keyed by a hash of the kernel source it was taken on; any
+# profiles/pair_gemm_kernel_qkv2048.md, keyed by a hash of the kernel source it was taken on; any
 # change to the kernel source makes the figure stale and it is reported as null.
-PROFILED_GEMM_TRAFFIC = {("qkv_2048", "e139ca2d2d9b"): 320.76e6}
+PROFILED_GEMM_TRAFFIC = {("qkv_2048", "5b52a0257f1d"): 49.85e6 + 258.10e6}
 # The same for kernel 1 (profiles/quant_act_kernel_qkv2048.md), keyed by a hash of its source.
-PROFILED_K1_TRAFFIC = {}
+PROFILED_K1_TRAFFIC = {("qkv_2048", "bcced91f73dc"): 104.06e6 + 6.44e6}
 
 
 def read_peaks():
@@ -189,14 +189,12 @@ def build_layers(wl, dev, lora=0):
     return layers
 
 
-def run_step(layers, ev=None, dynamic=False):
+def run_step(layers, dynamic=False):
     import bit_diffusion_transformer_svdquant_b200 as svdq
-    for i, L in enumerate(layers):
+    for L in layers:
         if dynamic:
             svdq.calibrate_act(L["X"], L["w"], out=L["g_x"])
         svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
-        if ev is not None:
-            ev[i].record()
         svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
 
 
@@ -231,6 +229,39 @@ def time_per_step(fn, steps, flush, stream, clean=None):
     return statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
 
 
+def two_pass(run, n_marks, K, flush, stream, dev, clean=None, wall=None):
+    """Times K steps of run(mark) twice under the L2-flush protocol (flush outside the events).
+
+    Pass 1 records events only at the step boundaries, with mark a no-op: the step time. An event
+    between two kernels on the stream costs a few microseconds of drain before the next launch and
+    keeps the next kernel from starting while the previous one finishes, so none is recorded there.
+    Pass 2 records an event at every mark(j), j = 0 .. n_marks - 1, which run calls after each of
+    its kernels: their durations. Returns (mean step ms of pass 1, [mean ms from the step start to
+    mark 0, from mark 0 to mark 1, ...] of pass 2, clock record of pass 1). With `wall` (a list),
+    the host wall time of pass 1 is appended to it."""
+    se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t0 = time.perf_counter()
+        for e0, e1 in se:
+            flush_l2(flush, clean)
+            e0.record(stream)
+            run(lambda j: None)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if wall is not None:
+            wall.append(time.perf_counter() - t0)
+    step_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in se)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks + 1)] for _ in range(K)]
+    for row in ev:
+        flush_l2(flush, clean)
+        row[0].record(stream)
+        run(lambda j, row=row: row[j + 1].record(stream))
+    torch.cuda.synchronize(dev)
+    parts = [statistics.mean(row[j].elapsed_time(row[j + 1]) for row in ev) for j in range(n_marks)]
+    return step_ms, parts, clk.summary()
+
+
 def gpu_arm(args, rank, world, dev):
     import bit_diffusion_transformer_svdquant_b200 as svdq
 
@@ -249,56 +280,32 @@ def gpu_arm(args, rank, world, dev):
 
     K = args.steps
     n_l = len(layers)
-    # Events per step: one at the start, then one after each kernel (the start of the next kernel
-    # is the end of the previous one). Every timing event on the stream costs a few microseconds
-    # of drain before the next launch (measured on B200), so no redundant ones are recorded.
-    # ev[s][0] = step start; per layer i: [1 + 3i] after the amax pass (dynamic mode only, else
-    # the same event as the layer start), [2 + 3i] after kernel 1, [3 + 3i] after the GEMM.
-    def new_ev():
-        return torch.cuda.Event(enable_timing=True)
-    ev = []
-    for _ in range(K):
-        row = [new_ev()]
-        for _ in range(n_l):
-            row += [new_ev() if dyn else None, new_ev(), new_ev()]
-        ev.append(row)
+    per = 3 if dyn else 2   # marks per layer: [after the amax pass,] after kernel 1, after the GEMM
+
+    def run(mark):
+        for i, L in enumerate(layers):
+            if dyn:
+                svdq.calibrate_act(L["X"], L["w"], out=L["g_x"])
+                mark(per * i)
+            svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
+            mark(per * i + per - 2)
+            svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
+            mark(per * i + per - 1)
 
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
-        t_wall = time.perf_counter()
-        for s in range(K):
-            flush_l2(flush, clean)
-            row = ev[s]
-            row[0].record(stream)
-            for i, L in enumerate(layers):
-                if dyn:
-                    svdq.calibrate_act(L["X"], L["w"], out=L["g_x"])
-                    row[1 + 3 * i].record(stream)
-                svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
-                row[2 + 3 * i].record(stream)
-                svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
-                row[3 + 3 * i].record(stream)
-        torch.cuda.synchronize(dev)
-        t_wall = time.perf_counter() - t_wall
+    wall = []
+    step_ms, parts, clocks = two_pass(run, per * n_l, K, flush, stream, dev, clean, wall)
     if world > 1:
         torch.distributed.barrier()
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out during the timed region")
-
-    def layer_start(row, i):
-        return row[0] if i == 0 else row[3 * i]
-
-    def k1_start(row, i):
-        return row[1 + 3 * i] if dyn else layer_start(row, i)
-
-    step_ms = [ev[s][0].elapsed_time(ev[s][3 * n_l]) for s in range(K)]
-    total_ms = float(sum(step_ms))
-    kc_ms = [[layer_start(ev[s], i).elapsed_time(ev[s][1 + 3 * i]) if dyn else 0.0 for s in range(K)]
-             for i in range(n_l)]
-    k1_ms = [[k1_start(ev[s], i).elapsed_time(ev[s][2 + 3 * i]) for s in range(K)] for i in range(n_l)]
-    k2_ms = [[ev[s][2 + 3 * i].elapsed_time(ev[s][3 + 3 * i]) for s in range(K)] for i in range(n_l)]
+    t_wall = wall[0]
+    total_ms = step_ms * K
+    kc_ms = [parts[per * i] if dyn else 0.0 for i in range(n_l)]
+    k1_ms = [parts[per * i + per - 2] for i in range(n_l)]
+    k2_ms = [parts[per * i + per - 1] for i in range(n_l)]
+    split_ms = sum(parts)
     total_ms = max_over_ranks(total_ms, dev)
 
     flops_main = sum(layer_flops(L["spec"])[0] for L in layers)
@@ -310,12 +317,12 @@ def gpu_arm(args, rank, world, dev):
     # dominant kernel: the GEMM of the largest layer
     big = max(range(n_l), key=lambda i: layer_flops(layers[i]["spec"])[0])
     spec_b = layers[big]["spec"]
-    k2_avg = statistics.mean(k2_ms[big])
+    k2_avg = k2_ms[big]
     peaks = read_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     gemm_flops = gemm_kernel_flops(spec_b)
     achieved = gemm_flops / (k2_avg * 1e-3) / 1e12
-    k1_avg = [statistics.mean(k1_ms[i]) for i in range(n_l)]
+    k1_avg = k1_ms
     k1_gbs = [kernel1_bytes(layers[i]["spec"]) / (k1_avg[i] * 1e-3) / 1e9 for i in range(n_l)]
     big1 = max(range(n_l), key=lambda i: kernel1_bytes(layers[i]["spec"]))
 
@@ -363,10 +370,11 @@ def gpu_arm(args, rank, world, dev):
             "quantize_act_us": [round(x * 1e3, 2) for x in k1_avg],
             "quantize_act_gbs": [round(x, 1) for x in k1_gbs],
             "quantize_act_frac_hbm": [round(x / peaks["hbm_gbs"], 4) for x in k1_gbs],
-            "gemm_us": [round(statistics.mean(k2_ms[i]) * 1e3, 2) for i in range(n_l)],
-            **({"dynamic_scale_us": [round(statistics.mean(kc_ms[i]) * 1e3, 2) for i in range(n_l)]} if dyn else {}),
+            "gemm_us": [round(k2_ms[i] * 1e3, 2) for i in range(n_l)],
+            "step_us_with_an_event_after_each_kernel": round(split_ms * 1e3, 2),
+            **({"dynamic_scale_us": [round(kc_ms[i] * 1e3, 2) for i in range(n_l)]} if dyn else {}),
         },
-        "roofline": {"bound": "tensor", "kernel": "svdq_gemm_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "tensor", "kernel": "pair_gemm_kernel<Nvfp4Gemm>", "achieved": round(achieved, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
                      "traffic": PROFILED_GEMM_TRAFFIC.get((wl.name, gemm_source_hash())),
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
@@ -391,7 +399,7 @@ def gpu_arm(args, rank, world, dev):
                                          "SwiGLU, same shapes",
                                  "speedup_of_this_path": round(base_ms / ms_per_step, 3)},
         "gpu_launches": (4 if dyn else 2) * n_l * K,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 3),
     }
     return out
@@ -516,16 +524,12 @@ def fp8r_arm(args, dev):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if args.l2_clean else None
 
-    def step(ev=None):
+    def step(mark=lambda j: None):
         for i, L in enumerate(layers):
-            if ev is not None:
-                ev[i][0].record(stream)
             svdq.quantize_act_fp8r(L["X"], L["w"], L["act"])
-            if ev is not None:
-                ev[i][1].record(stream)
+            mark(2 * i)
             svdq.gemm_fp8r(L["act"], L["w"], L["bias"], out=L["Y"])
-            if ev is not None:
-                ev[i][2].record(stream)
+            mark(2 * i + 1)
 
     for _ in range(args.warmup):
         step()
@@ -533,26 +537,16 @@ def fp8r_arm(args, dev):
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out during the FP8 warm-up")
     K, n_l = args.steps, len(layers)
-    se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    kev = [[tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_l)] for _ in range(K)]
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
-        for s in range(K):
-            flush_l2(flush, clean)
-            se[s][0].record(stream)
-            step(kev[s])
-            se[s][1].record(stream)
-        torch.cuda.synchronize(dev)
+    ms, parts, clocks = two_pass(step, 2 * n_l, K, flush, stream, dev, clean)
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out in the FP8 timed region")
-    ms = statistics.mean(a.elapsed_time(b) for a, b in se)
-    k1 = [statistics.mean(kev[s][i][0].elapsed_time(kev[s][i][1]) for s in range(K)) for i in range(n_l)]
-    k2 = [statistics.mean(kev[s][i][1].elapsed_time(kev[s][i][2]) for s in range(K)) for i in range(n_l)]
+    k1 = [parts[2 * i] for i in range(n_l)]
+    k2 = [parts[2 * i + 1] for i in range(n_l)]
     flops_main = sum(layer_flops(L["spec"])[0] for L in layers)
     big = max(range(n_l), key=lambda i: layer_flops(layers[i]["spec"])[0])
     peaks = read_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
-    achieved = sum(layer_flops(layers[big]["spec"])) / (k2[big] * 1e-3) / 1e12
+    achieved = gemm_kernel_flops(layers[big]["spec"]) / (k2[big] * 1e-3) / 1e12
     rel = []
     for L in layers:
         rows = min(256, L["spec"].M)
@@ -567,13 +561,15 @@ def fp8r_arm(args, dev):
             "steps": K, "warmup": args.warmup, "dtype": "fp8 e4m3 row-wise + bf16 low-rank, fp32 acc",
             "kernels": {"quantize_act_us": [round(x * 1e3, 2) for x in k1],
                         "gemm_us": [round(x * 1e3, 2) for x in k2]},
-            "roofline": {"bound": "tensor", "kernel": "fp8r::gemm_kernel", "achieved": round(achieved, 1),
+            "roofline": {"bound": "tensor", "kernel": "pair_gemm_kernel<Fp8Gemm>", "achieved": round(achieved, 1),
                          "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
                          "traffic": None,
                          "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
-                                        f"{FP8_PER_BF16} (nominal dense FP8/bf16 ratio)"},
+                                        f"{FP8_PER_BF16} (nominal dense FP8/bf16 ratio)",
+                         "algorithmic": f"{gemm_kernel_flops(layers[big]['spec']) / 1e9:.1f} GFLOP per launch "
+                                        "(2MNK + 2MrN)"},
             "rel_err_vs_unquantized_first_rows": rel,
-            "gpu_launches": 3 * n_l * K, "clocks": clk.summary(),
+            "gpu_launches": 3 * n_l * K, "clocks": clocks,
             "what": "the same workload through the row-wise FP8 kernels (row-scale pass, quantizing pass, "
                     "kind::f8f6f4 GEMM), run in a separate process"}
 
@@ -601,18 +597,13 @@ def mlp_fused_arm(args, dev):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if args.l2_clean else None
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def step(mark=lambda j: None):
         svdq.quantize_act(up["X"], up["w"], up["g_x"], up["act"])
-        if ev is not None:
-            ev[1].record(stream)
+        mark(0)
         svdq.gemm_swiglu_quant(up["act"], up["w"], up["bias"], dn["w"], dn["g_x"], act_dn, scratch)
-        if ev is not None:
-            ev[2].record(stream)
+        mark(1)
         svdq.gemm(act_dn, dn["w"], dn["bias"], out=Y)
-        if ev is not None:
-            ev[3].record(stream)
+        mark(2)
 
     for _ in range(args.warmup):
         step()
@@ -625,17 +616,9 @@ def mlp_fused_arm(args, dev):
     ref = dn["Y"].float()
     diff = float((Y.float() - ref).norm() / ref.norm())
     K = args.steps
-    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
-        for s in range(K):
-            flush_l2(flush, clean)
-            step(ev[s])
-        torch.cuda.synchronize(dev)
+    ms, part, clocks = two_pass(step, 3, K, flush, stream, dev, clean)
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out in the fused timed region")
-    ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
-    part = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(3)]
     # the unfused chain (kernel 1 + GEMM per layer, h through HBM) under the same protocol
     unf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for s in range(K):
@@ -653,7 +636,7 @@ def mlp_fused_arm(args, dev):
             "steps": K, "warmup": args.warmup,
             "kernels_us": {"quantize_act_up": round(part[0] * 1e3, 2), "gemm_swiglu_quant": round(part[1] * 1e3, 2),
                            "gemm_down": round(part[2] * 1e3, 2)},
-            "rel_diff_vs_unfused_chain": round(diff, 7), "gpu_launches": 4 * K, "clocks": clk.summary(),
+            "rel_diff_vs_unfused_chain": round(diff, 7), "gpu_launches": 4 * K, "clocks": clocks,
             "what": "gate/up GEMM with the down layer's kernel 1 fused into its SwiGLU epilogue, then the down "
                     "GEMM; run in a separate process"}
 
@@ -670,22 +653,19 @@ def config_row_arm(args, dev):
         run_step(layers)
     torch.cuda.synchronize(dev)
     K, n_l = args.steps, len(layers)
-    ev = [[tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_l)] for _ in range(K)]
-    for s_ in range(K):
-        flush_l2(flush)
+
+    def run(mark):
         for i, L in enumerate(layers):
-            e0, e1, e2 = ev[s_][i]
-            e0.record(stream)
             svdq.quantize_act(L["X"], L["w"], L["g_x"], L["act"])
-            e1.record(stream)
+            mark(2 * i)
             svdq.gemm(L["act"], L["w"], L["bias"], out=L["Y"])
-            e2.record(stream)
-    torch.cuda.synchronize(dev)
+            mark(2 * i + 1)
+
+    ms, parts, _ = two_pass(run, 2 * n_l, K, flush, stream, dev)
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out")
-    ms = statistics.mean(ev[s_][0][0].elapsed_time(ev[s_][-1][2]) for s_ in range(K))
-    k1 = [statistics.mean(ev[s_][i][0].elapsed_time(ev[s_][i][1]) for s_ in range(K)) for i in range(n_l)]
-    k2 = [statistics.mean(ev[s_][i][1].elapsed_time(ev[s_][i][2]) for s_ in range(K)) for i in range(n_l)]
+    k1 = [parts[2 * i] for i in range(n_l)]
+    k2 = [parts[2 * i + 1] for i in range(n_l)]
     peaks = read_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     flops = sum(layer_flops(L["spec"])[0] for L in layers)

@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <string>
 
 #include "svdq.h"
@@ -326,6 +327,30 @@ svdq_status check_launch(const char* what) {
   return SVDQ_OK;
 }
 
+// Both kernels of a layer are launched with programmatic stream serialization: a kernel may be
+// scheduled while the previous kernel on the stream is finishing, so its barrier and TMEM set-up
+// overlap that kernel's tail; its first global access waits for that grid (griddepcontrol.wait).
+void set_programmatic(cudaLaunchAttribute& a) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+}
+
+// The pair GEMMs: clusters of 2 CTAs are compiled into the kernel, so the one launch attribute is
+// the programmatic one.
+template <typename... P, typename... A>
+cudaError_t launch_pair_gemm(void (*kern)(P...), int ctas, int smem, cudaStream_t st, A&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  set_programmatic(attr[0]);
+  cfg.gridDim = dim3(ctas, 1, 1);
+  cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 }  // namespace
 
 extern "C" {
@@ -527,16 +552,17 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
   a.k_per_cta = K / csize;
 
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  set_programmatic(attr[1]);
   cfg.gridDim = dim3(m_tiles * csize, 1, 1);
   cfg.blockDim = dim3(svdq::kQ1Threads, 1, 1);
   cfg.stream = static_cast<cudaStream_t>(stream);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaSuccess;
   switch (r) {
     case 0:
@@ -628,18 +654,18 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
     max_pairs = g_dev[dev].max_pairs[n_tile == 256 ? 0 : n_tile == 192 ? 1 : 2];
   }
   const int pairs = g.num_tiles < max_pairs ? g.num_tiles : max_pairs;
-  const dim3 grid(2 * pairs);  // clusters of 2 CTAs (compiled into the kernel)
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (n_tile == 256) {
-    svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 256, kStagesTile256><<<grid, svdq::kGemmThreads, svdq::GemmLayout<256, kStagesTile256>::kSmem, st>>>(
-        tmA, tmB, tmU, tmL2, tmY, g);
-  } else if (n_tile == 192) {
-    svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 192, kStagesTile192><<<grid, svdq::kGemmThreads, svdq::GemmLayout<192, kStagesTile192>::kSmem, st>>>(
-        tmA, tmB, tmU, tmL2, tmY, g);
-  } else {
-    svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 128, kStagesTile128><<<grid, svdq::kGemmThreads, svdq::GemmLayout<128, kStagesTile128>::kSmem, st>>>(
-        tmA, tmB, tmU, tmL2, tmY, g);
-  }
+  cudaError_t e;
+  if (n_tile == 256)
+    e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 256, kStagesTile256>, 2 * pairs,
+                         svdq::GemmLayout<256, kStagesTile256>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
+  else if (n_tile == 192)
+    e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 192, kStagesTile192>, 2 * pairs,
+                         svdq::GemmLayout<192, kStagesTile192>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
+  else
+    e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 128, kStagesTile128>, 2 * pairs,
+                         svdq::GemmLayout<128, kStagesTile128>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of pair_gemm_kernel failed: %s", cudaGetErrorString(e));
   return check_launch("pair_gemm_kernel (NVFP4)");
 }
 
@@ -968,16 +994,17 @@ svdq_status svdq_fp8r_quantize_act(const uint16_t* X, const svdq_fp8r_weight* w,
   a.k_per_cta = K / csize;
 
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  set_programmatic(attr[1]);
   cfg.gridDim = dim3(m_tiles * csize, 1, 1);
   cfg.blockDim = dim3(svdq::kQ1Threads, 1, 1);
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaSuccess;
   switch (r) {
     case 0:
@@ -1068,18 +1095,18 @@ svdq_status svdq_fp8r_gemm(const svdq_fp8r_act* act, const svdq_fp8r_weight* w, 
     max_pairs = g_fp8r[dev].max_pairs[n_tile == 256 ? 0 : n_tile == 192 ? 1 : 2];
   }
   const int pairs = g.num_tiles < max_pairs ? g.num_tiles : max_pairs;
-  const dim3 grid(2 * pairs);  // clusters of 2 CTAs (compiled into the kernel)
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (n_tile == 256) {
-    svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 256, kFp8Stages256>
-        <<<grid, svdq::kGemmThreads, svdq::PairGemmLayout<false, 256, kFp8Stages256>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
-  } else if (n_tile == 192) {
-    svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 192, kFp8Stages192>
-        <<<grid, svdq::kGemmThreads, svdq::PairGemmLayout<false, 192, kFp8Stages192>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
-  } else {
-    svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 128, kFp8Stages128>
-        <<<grid, svdq::kGemmThreads, svdq::PairGemmLayout<false, 128, kFp8Stages128>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmY, g);
-  }
+  cudaError_t e;
+  if (n_tile == 256)
+    e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 256, kFp8Stages256>, 2 * pairs,
+                         svdq::PairGemmLayout<false, 256, kFp8Stages256>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
+  else if (n_tile == 192)
+    e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 192, kFp8Stages192>, 2 * pairs,
+                         svdq::PairGemmLayout<false, 192, kFp8Stages192>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
+  else
+    e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::fp8r::Fp8Gemm, 128, kFp8Stages128>, 2 * pairs,
+                         svdq::PairGemmLayout<false, 128, kFp8Stages128>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of pair_gemm_kernel failed: %s", cudaGetErrorString(e));
   return check_launch("pair_gemm_kernel (row-wise FP8)");
 }
 

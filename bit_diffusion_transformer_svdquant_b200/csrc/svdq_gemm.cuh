@@ -246,6 +246,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
+  // The set-up above touches no global memory, so it overlaps the end of the previous kernel on the
+  // stream (programmatic launch); everything below may read what that kernel wrote.
+  grid_dependency_wait();
+  grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   unsigned* status = &g_svdq_status;
   const uint64_t wait_ns = args.wait_ns;

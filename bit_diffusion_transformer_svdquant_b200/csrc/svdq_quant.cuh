@@ -313,8 +313,10 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   unsigned* status = &g_svdq_status;
   const uint64_t wait_ns = a.wait_ns;
 
-  // the first ring fill (one load per slot) is issued by the producer thread right after the barrier
-  // set-up, so its latency overlaps the TMEM allocation and the table set-up of the other warps
+  // Barrier set-up and the TMEM allocation touch no global memory, so they run before the wait for
+  // the previous kernel on the stream (which may still be finishing: programmatic launch). The
+  // first ring fill (one load per slot) is then issued by the producer thread at once, so its
+  // latency overlaps the table set-up of the other warps.
   const int n_pre = n_steps < S ? n_steps : S;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -326,6 +328,14 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
+  }
+  if (R > 0 && warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (threadIdx.x == 0) {
     const uint64_t pol_x = l2_policy_evict_first();
     for (int st = 0; st < n_pre; ++st) {
       const uint32_t sa = sbase + st * L::kStage;
@@ -335,10 +345,6 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       if (R > 0) tma_load_2d(sa + kQTile, &tmL1, kx, 0, full_bar(st));
       bulk_load(sa + L::kLamOff, a.inv_lambda + kx, 256, full_bar(st));
     }
-  }
-  if (R > 0 && warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), L::kTmemCols);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
