@@ -958,8 +958,21 @@ svdq_status svdq_fp8r_quantize_act(const uint16_t* X, const svdq_fp8r_weight* w,
   const int K = act->K, r = w->r, M = act->M;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // row scales first: the quantizing pass needs each row's amax before its first code
-  svdq::fp8r::act_row_scale_kernel<<<grid_for(static_cast<size_t>(act->M_pad) * 32, 256, sms), 256, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(X), w->inv_lambda, M, act->M_pad, K, act->row_scale, act->row_rscale);
+  {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    set_programmatic(attr[0]);
+    cfg.gridDim = dim3(grid_for(static_cast<size_t>(act->M_pad) * 32, 256, sms), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e =
+        cudaLaunchKernelEx(&cfg, svdq::fp8r::act_row_scale_kernel, reinterpret_cast<const __nv_bfloat16*>(X),
+                           static_cast<const float*>(w->inv_lambda), M, act->M_pad, K, act->row_scale, act->row_rscale);
+    if (e != cudaSuccess)
+      return fail(SVDQ_ERR_CUDA, "launch of fp8r::act_row_scale_kernel failed: %s", cudaGetErrorString(e));
+  }
   if (svdq_status s = check_launch("fp8r::act_row_scale_kernel"); s != SVDQ_OK) return s;
   CUtensorMap tmX, tmL1;
   std::memset(&tmL1, 0, sizeof(tmL1));
@@ -1292,28 +1305,38 @@ svdq_status svdq_gemm_swiglu_quant(const svdq_act* act, const svdq_weight* w, co
   a.num_units = a.m_pairs * splits;
   const int pairs = a.num_units < max_pairs ? a.num_units : max_pairs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const dim3 grid(2 * pairs);
+  cudaError_t e;
   switch (r2) {
     case 16:
-      svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 16>
-          <<<grid, svdq::kGemmThreads, svdq::fused::Layout<kFusedStages, 16>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmH,
-                                                                                          tmL1n, a);
+      e = launch_pair_gemm(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 16>, 2 * pairs,
+                           svdq::fused::Layout<kFusedStages, 16>::kSmem, st, tmA, tmB, tmU, tmL2, tmH, tmL1n, a);
       break;
     case 32:
-      svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 32>
-          <<<grid, svdq::kGemmThreads, svdq::fused::Layout<kFusedStages, 32>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmH,
-                                                                                          tmL1n, a);
+      e = launch_pair_gemm(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 32>, 2 * pairs,
+                           svdq::fused::Layout<kFusedStages, 32>::kSmem, st, tmA, tmB, tmU, tmL2, tmH, tmL1n, a);
       break;
     default:
-      svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 64>
-          <<<grid, svdq::kGemmThreads, svdq::fused::Layout<kFusedStages, 64>::kSmem, st>>>(tmA, tmB, tmU, tmL2, tmH,
-                                                                                          tmL1n, a);
+      e = launch_pair_gemm(svdq::fused::gemm_swiglu_quant_kernel<kFusedStages, 64>, 2 * pairs,
+                           svdq::fused::Layout<kFusedStages, 64>::kSmem, st, tmA, tmB, tmU, tmL2, tmH, tmL1n, a);
       break;
   }
+  if (e != cudaSuccess)
+    return fail(SVDQ_ERR_CUDA, "launch of fused::gemm_swiglu_quant_kernel failed: %s", cudaGetErrorString(e));
   if (svdq_status s = check_launch("fused::gemm_swiglu_quant_kernel"); s != SVDQ_OK) return s;
-  svdq::fused::finalize_u_kernel<<<grid_for(static_cast<size_t>(act_next->M_pad) * r2, 256, sms), 256, 0, st>>>(
-      static_cast<const float*>(scratch), splits, act->M, act_next->M_pad, r2, g_x_next, w_next->g_w,
-      static_cast<__nv_bfloat16*>(act_next->U), act_next->alpha);
+  {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    set_programmatic(attr[0]);
+    cfg.gridDim = dim3(grid_for(static_cast<size_t>(act_next->M_pad) * r2, 256, sms), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, svdq::fused::finalize_u_kernel, static_cast<const float*>(scratch), splits, act->M,
+                           act_next->M_pad, r2, g_x_next, static_cast<const float*>(w_next->g_w),
+                           static_cast<__nv_bfloat16*>(act_next->U), act_next->alpha);
+  }
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "launch of fused::finalize_u_kernel failed: %s", cudaGetErrorString(e));
   return check_launch("fused::finalize_u_kernel");
 }
 

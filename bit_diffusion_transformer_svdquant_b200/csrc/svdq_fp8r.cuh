@@ -14,10 +14,10 @@
 // three bf16 MMAs per 16 columns of r (hi.hi, lo.hi, hi.lo) add U L2 / (s_x s_w) before the
 // epilogue multiplies every accumulator element by s_x[m] s_w[n].
 //
-// Kernels: pack_weight_kernel / pack_l2_kernel (offline), act_row_scale_kernel and
-// quant_act_kernel (per call, the latter the NVFP4 kernel 1's TMA + tcgen05 structure with a
-// per-element E4M3 quantizer), gemm_kernel (the NVFP4 GEMM's CTA-pair structure with
-// tcgen05.mma kind::f8f6f4, no scale-factor operands, double-buffered accumulators).
+// Kernels: pack_weight_kernel / pack_l2_kernel (offline); per call act_row_scale_kernel, then kernel 1
+// (svdq::quant_act_kernel) with the RowAct quantizer policy below (a per-element E4M3 quantizer),
+// then the pair GEMM (svdq::pair_gemm_kernel) with the Fp8Gemm format policy below (tcgen05.mma
+// kind::f8f6f4, no scale-factor operands, double-buffered accumulators).
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -128,6 +128,8 @@ __global__ void export_weight_kernel(const uint8_t* __restrict__ codes, const fl
 // rs_x[m] = fp32(1 / s_x[m]); pad rows M <= m < M_pad get 1. One warp per row, 16-byte loads.
 __global__ void act_row_scale_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ inv_lambda,
                                      int M, int M_pad, int K, float* __restrict__ s_x, float* __restrict__ rs_x) {
+  grid_dependency_wait();  // X (and the row scales the previous call's GEMM read) belong to earlier kernels
+  grid_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
   for (int m = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); m < M_pad; m += warps) {

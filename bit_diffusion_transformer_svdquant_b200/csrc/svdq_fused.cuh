@@ -171,11 +171,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       prefetch_tmap(&tmL2);
     }
   }
-  // the next layer's reciprocal-scale table, as kernel 1 builds it
-  if (threadIdx.x < 128) {
-    const float gx2 = *args.g_x2;
-    reinterpret_cast<float*>(smem + L::kTabOff)[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_value(threadIdx.x), gx2));
-  }
   if (warp == 1) {
     tmem_alloc_pair(smem_addr(tmem_slot), 512);
     tmem_relinquish_pair();
@@ -184,6 +179,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
+  // The set-up above touches no global memory, so it overlaps the end of the previous kernel on the
+  // stream (programmatic launch); everything below may read what that kernel wrote.
+  grid_dependency_wait();
+  grid_launch_dependents();
+  // the next layer's reciprocal-scale table, as kernel 1 builds it
+  if (threadIdx.x < 128) {
+    const float gx2 = *args.g_x2;
+    reinterpret_cast<float*>(smem + L::kTabOff)[threadIdx.x] = __frcp_rn(__fmul_rn(e4m3_value(threadIdx.x), gx2));
+  }
+  __syncthreads();
   const uint32_t tmem = *tmem_slot;
   unsigned* status = &g_svdq_status;
   const uint64_t wait_ns = args.wait_ns;
@@ -618,6 +623,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 __global__ void finalize_u_kernel(const float* __restrict__ partials, int splits, int M, int M_pad, int r,
                                   const float* g_x2, const float* g_w2, __nv_bfloat16* __restrict__ U,
                                   float* alpha_out) {
+  grid_dependency_wait();  // the partial sums of the kernel before it on the stream
+  grid_launch_dependents();
   const float alpha = __fmul_rn(*g_x2, *g_w2);
   const float cinv = __frcp_rn(alpha);
   const size_t total = static_cast<size_t>(M_pad) * r;
