@@ -31,6 +31,9 @@
  *   - Work is enqueued on `stream` (a cudaStream_t / CUstream; NULL = legacy default stream) and is
  *     asynchronous; argument checks happen on the host before anything is enqueued, and on a
  *     failed check nothing is enqueued.
+ *   - The per-call kernels are launched with programmatic stream serialization: one may start its
+ *     set-up (barriers, tensor memory) while the kernel before it on the stream is finishing, but
+ *     it reads or writes no global memory until that kernel has completed. Stream order is kept.
  *   - Shapes: K % 256 == 0; N % n_tile == 0 for the n_tile chosen at pack time (256 where it
  *     divides N, else 192, else 128; SwiGLU needs N even); r in {0, 16, 32, 64}; 1 <= M < 2^24.
  *     Device pointers 16-byte aligned.
