@@ -50,7 +50,7 @@ struct DeviceState {
   bool ready = false;
   int sm_count = 0;
   int max_pairs[3] = {0, 0, 0};  // co-resident CTA pairs of the GEMM kernel for n_tile 256, 192, 128
-  int k1_clusters[4][3] = {};     // co-resident kernel-1 clusters, by r (0/16/32/64) and size (1/2/4)
+  int k1_clusters[4][4] = {};     // co-resident kernel-1 clusters, by r (0/16/32/64) and size - 1 (1..4)
   svdq_status status = SVDQ_OK;
   std::string error;
 };
@@ -130,10 +130,11 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
                                   svdq::GemmLayout<128, kStagesTile128>::kSmem, &st.max_pairs[2]);
         s != SVDQ_OK)
       return s;
-    // how many kernel-1 clusters of 1, 2 and 4 CTAs (one CTA per SM) can be resident at once
+    // how many kernel-1 clusters of 1, 2, 3 and 4 CTAs (one CTA per SM) can be resident at once
+    // (a cluster's CTAs share a GPC, so fewer 4-clusters than sms / 4 may fit)
     auto k1_clusters = [&](const void* fn, int smem, int* out) -> svdq_status {
-      for (int ci = 0; ci < 3; ++ci) {
-        const int c = 1 << ci;
+      for (int ci = 0; ci < 4; ++ci) {
+        const int c = ci + 1;
         cudaLaunchConfig_t cfg{};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -521,21 +522,23 @@ svdq_status svdq_quantize_act(const uint16_t* X, const svdq_weight* w, const flo
         s != SVDQ_OK)
       return s;
   }
-  // One CTA per SM; K is split across a cluster of 2 or 4 CTAs only while all row tiles' clusters
-  // of that size are resident at once (cudaOccupancyMaxActiveClusters: clusters must fit inside
-  // GPCs), so small M fills more SMs and nothing runs as a second wave. SVDQ_K1_CLUSTER overrides
-  // the size; every CTA keeps whole 64-column K steps.
+  // One CTA per SM; K is split across the largest cluster of 2, 3 or 4 CTAs whose clusters for all
+  // row tiles are resident at once (cudaOccupancyMaxActiveClusters: clusters must fit inside GPCs),
+  // so small M fills more SMs and nothing runs as a second wave. Measured on B200 at M = 4608 (36 row
+  // tiles): only 32 clusters of 4 are resident, and at K = 12288 3-CTA clusters (108 CTAs) take
+  // 47 us against 57 us for 2-CTA ones (72 CTAs). SVDQ_K1_CLUSTER overrides the size; every CTA
+  // keeps whole 64-column K steps.
   const int m_tiles = act->M_pad / 128;
   int csize = 1;
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     const int* mc = g_dev[dev].k1_clusters[r == 0 ? 0 : r == 16 ? 1 : r == 32 ? 2 : 3];
-    if (m_tiles <= mc[1] && (K / 2) % 64 == 0) csize = 2;
-    if (m_tiles <= mc[2] && (K / 4) % 64 == 0) csize = 4;
+    for (int c = 2; c <= 4; ++c)
+      if (m_tiles <= mc[c - 1] && K % (64 * c) == 0) csize = c;
   }
   if (const char* env = getenv("SVDQ_K1_CLUSTER"); env != nullptr) {
     const int c = atoi(env);
-    if ((c == 1 || c == 2 || c == 4) && (K / c) % 64 == 0) csize = c;
+    if (c >= 1 && c <= 4 && K % (64 * c) == 0) csize = c;
   }
   svdq::QuantActArgs a;
   a.inv_lambda = w->inv_lambda;
@@ -992,8 +995,8 @@ svdq_status svdq_fp8r_quantize_act(const uint16_t* X, const svdq_fp8r_weight* w,
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     const int* mc = g_dev[dev].k1_clusters[r == 0 ? 0 : r == 16 ? 1 : r == 32 ? 2 : 3];
-    if (m_tiles <= mc[1] && (K / 2) % 64 == 0) csize = 2;
-    if (m_tiles <= mc[2] && (K / 4) % 64 == 0) csize = 4;
+    for (int c = 2; c <= 4; ++c)
+      if (m_tiles <= mc[c - 1] && K % (64 * c) == 0) csize = c;
   }
   svdq::fp8r::ActArgs a;
   a.inv_lambda = w->inv_lambda;
