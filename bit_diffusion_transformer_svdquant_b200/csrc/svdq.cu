@@ -1157,7 +1157,7 @@ svdq_status svdq_fp8r_export_act(const svdq_fp8r_act* act, uint8_t* codes, float
 // ================================================================== MLP chain: kernel 1 fused into SwiGLU
 namespace {
 
-constexpr int kFusedStages = 4;
+constexpr int kFusedStages = 5;
 constexpr int kMaxSplits = 8;
 
 struct FusedState {

@@ -18,8 +18,10 @@
 //   schedule   units of (256-row block, column split): a pair sweeps the split's column tiles of one
 //              row block in order, so U' accumulates in its TMEM; splits are chosen so that the
 //              units about fill the resident pairs;
-//   producer   after a tile's K steps, that tile's L1s'^T slice (r/2 rows per CTA x 128 columns,
-//              two 128B-swizzled boxes) into one of two slice buffers;
+//   producer   after a tile's K steps, the PREVIOUS tile's L1s'^T slice (r/2 rows per CTA x 128
+//              columns, two 128B-swizzled boxes) into the next ring slot, so that no slice buffer
+//              takes the shared memory of a fifth ring stage (the writers report that slot like a
+//              low-rank slot, and the U' MMAs that read it release it);
 //   issuer     after tile t's K loop it issues the U' MMAs of tile t-1 (the epilogue of t-1 ran
 //              meanwhile), then the accumulator commit of t; the unit's first U' MMA overwrites
 //              the U' accumulator once the previous unit's has been drained;
@@ -28,9 +30,8 @@
 //              accumulator is released the h tile is read back and quantized for the next layer;
 //              at the end of a unit four warps per CTA drain U' into the partials buffer.
 // Barriers added to the GEMM's, each completing once per use in an order that no waiter can fall
-// two phases behind: lf_full[2] (slice landed, per CTA), slice_empty[2] (slice read by its U' MMAs),
-// h_full (both CTAs' h tiles written and their slices landed; the even CTA's), h_empty (the h tile
-// read), u_done (a unit's U' complete), u_free (a unit's U' drained; the even CTA's).
+// two phases behind: h_full (both CTAs' h tiles written; the even CTA's), h_empty (the h tile read),
+// u_done (a unit's U' complete), u_free (a unit's U' drained; the even CTA's).
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -75,20 +76,20 @@ struct Layout {
   static constexpr int kStage = G::kStage;
   static constexpr int kHTile = 128 * 128 * 2;        // 128 rows x 128 bf16: two 64-column atoms
   static constexpr int kHOff = STAGES * kStage;
-  static constexpr int kSliceAtom = (R2 / 2) * 128;   // r/2 rows of L1s'^T x 64 bf16 columns
+  // a tile's L1s'^T slice (r/2 rows x 128 bf16 columns per CTA, two 64-column atoms) travels in a
+  // ring slot of its own, right before the U' MMAs that read it
+  static constexpr int kSliceAtom = (R2 / 2) * 128;
   static constexpr int kSlice = 2 * kSliceAtom;
-  static constexpr int kSliceOff = kHOff + kHTile;
-  static constexpr int kTabOff = kSliceOff + 2 * kSlice;  // 128 fp32: 1 / (dec(s) g_x') per scale code
+  static constexpr int kTabOff = kHOff + kHTile;  // 128 fp32: 1 / (dec(s) g_x') per scale code
   static constexpr int kBarOff = kTabOff + 512;
-  // full[S], empty[S], accf, acce, drain, sf_full[4], lf_full[2], slice_empty[2], h_full, h_empty,
-  // u_done, u_free
-  static constexpr int kNumBars = 2 * STAGES + 3 + G::kSfBufs + 8;
+  // full[S], empty[S], accf, acce, drain, sf_full[4], h_full, h_empty, u_done, u_free
+  static constexpr int kNumBars = 2 * STAGES + 3 + G::kSfBufs + 4;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
   static constexpr int kColU = G::kColSf + G::kSfBufs * G::kSfCols;  // U' accumulator columns
   static_assert(G::kAccBufs == 1, "one 256-column accumulator");
   static_assert(kColU + R2 <= 512, "TMEM budget");
-  static_assert(kHOff % 1024 == 0 && kSliceOff % 1024 == 0 && kSliceAtom % 1024 == 0,
-                "128B-swizzled tiles start on 1024-byte boundaries");
+  static_assert(kHOff % 1024 == 0 && kSliceAtom % 1024 == 0, "128B-swizzled tiles start on 1024-byte boundaries");
+  static_assert(kSlice <= kStage, "a slice fits a ring stage");
   static_assert(G::kSfBufs <= STAGES, "a scale buffer's previous slot must still own its ring stage");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
@@ -127,16 +128,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t acce_bar = accf_bar + 8u;
   const uint32_t drain_bar = accf_bar + 16u;
   auto sf_full_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 3 + b); };
-  auto lf_full_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 3 + kSfBufs + b); };
-  auto slice_empty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 3 + kSfBufs + 2 + b); };
-  const uint32_t h_full_bar = bar0 + 8u * (2 * STAGES + 3 + kSfBufs + 4);
+  const uint32_t h_full_bar = bar0 + 8u * (2 * STAGES + 3 + kSfBufs);
   const uint32_t h_empty_bar = h_full_bar + 8u;
   const uint32_t u_done_bar = h_full_bar + 16u;
   const uint32_t u_free_bar = h_full_bar + 24u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t h_tile = sbase + L::kHOff;
-  auto slice_buf = [&](int b) { return sbase + L::kSliceOff + static_cast<uint32_t>(b * L::kSlice); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = args.r;
@@ -152,10 +150,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     mbar_init(acce_bar, 16);  // 8 epilogue warps in each CTA
     mbar_init(drain_bar, 1);
     for (int b = 0; b < kSfBufs; ++b) mbar_init(sf_full_bar(b), 8);  // 4 writer warps in each CTA
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(lf_full_bar(b), 1);
-      mbar_init(slice_empty_bar(b), 1);
-    }
     mbar_init(h_full_bar, 16);  // 8 epilogue warps in each CTA
     mbar_init(h_empty_bar, 1);
     mbar_init(u_done_bar, 1);
@@ -197,18 +191,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, armed = 0, armed_parity = 0, lf_armed = 0, lf_parity = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
       const int rc = r < kLrChunk ? r : kLrChunk;
       const uint32_t lr_bytes = static_cast<uint32_t>((2 * 128 + G::kBRows) * rc * 2);
       const int sf_row_stride = args.K >> 6;
-      int tseq = 0;
+      const int y_slice = static_cast<int>(rank) * (R2 / 2);
+      int prev_n_blk = -1;  // the tile whose U' MMAs come next (after this tile's K steps)
       bool ok = true;
+      // the L1s'^T slice of tile `nb` (next-layer K columns nb*128 .. +127, this CTA's r/2 rows) into
+      // the next ring slot, which its U' MMAs read and release
+      auto load_slice = [&](int nb) -> bool {
+        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)) return false;
+        const uint32_t sa = sbase + stage * L::kStage;
+        mbar_arrive_expect_tx(full_bar(stage), L::kSlice);
+        tma_load_2d(sa, &tmL1n, nb * kHalf, y_slice, full_bar(stage));
+        tma_load_2d(sa + L::kSliceAtom, &tmL1n, nb * kHalf + 64, y_slice, full_bar(stage));
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        return true;
+      };
       for (int unit = pair0; ok && unit < args.num_units; unit += npairs) {
         int m_pair, split, n_beg, n_end;
         unit_range(unit, args.splits, args.n_tiles, m_pair, split, n_beg, n_end);
         const int m_blk = 2 * m_pair + static_cast<int>(rank);
         const int m_sf = m_blk < args.m_tiles ? m_blk : args.m_tiles - 1;
-        for (int n_blk = n_beg; ok && n_blk < n_end; ++n_blk, ++tseq) {
+        for (int n_blk = n_beg; ok && n_blk < n_end; ++n_blk) {
           const int b_row = n_blk * N_TILE + static_cast<int>(rank) * G::kBRows;
           for (int c0 = 0; c0 < r; c0 += kLrChunk) {
             if (!(ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, wait_ns, status, kStatusProducer, abort_flag)))
@@ -240,27 +248,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
           if (!ok) break;
-          // the tile's L1s'^T slice (next-layer K columns n_blk*128 .. +127, this CTA's r/2 rows)
-          // into buffer tseq % 2, once the U' MMAs of tile tseq - 2 have read that buffer
-          const int b = tseq & 1, use = tseq >> 1;
-          if (use > 0 && !(ok = mbar_wait_bounded(slice_empty_bar(b), static_cast<uint32_t>(use - 1) & 1u, wait_ns,
-                                                  status, kStatusProducer, abort_flag)))
-            break;
-          mbar_arrive_expect_tx(lf_full_bar(b), L::kSlice);
-          const int y = static_cast<int>(rank) * (R2 / 2);
-          tma_load_2d(slice_buf(b), &tmL1n, n_blk * kHalf, y, lf_full_bar(b));
-          tma_load_2d(slice_buf(b) + L::kSliceAtom, &tmL1n, n_blk * kHalf + 64, y, lf_full_bar(b));
-          lf_armed |= 1u << b;
-          lf_parity = (lf_parity & ~(1u << b)) | ((static_cast<uint32_t>(use) & 1u) << b);
+          // the previous tile's slice, for the U' MMAs the issuer adds after this tile's K steps
+          if (prev_n_blk >= 0 && !(ok = load_slice(prev_n_blk))) break;
+          prev_n_blk = n_blk;
         }
       }
+      if (ok && prev_n_blk >= 0) load_slice(prev_n_blk);
       // Drain: every copy this thread started has landed before the CTA may exit.
       for (int s = 0; s < STAGES; ++s)
         if (armed & (1u << s))
           mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, wait_ns, status, kStatusDrain, nullptr);
-      for (int b = 0; b < 2; ++b)
-        if (lf_armed & (1u << b))
-          mbar_wait_bounded(lf_full_bar(b), (lf_parity >> b) & 1u, wait_ns, status, kStatusDrain, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
@@ -286,14 +283,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int pend = -1;
       bool pend_first = false, pend_last = false;
       bool ok = true;
-      // U' += h(t) L1s'(t): A = the h tile (two 64-column atoms, 128 rows per CTA), B = slice t % 2
+      // U' += h(t) L1s'(t): A = the h tile (two 64-column atoms, 128 rows per CTA), B = tile t's slice
+      // in the next ring slot (both CTAs' halves landed once the slot's sf_full completes)
       auto issue_u = [&](int t, bool first, bool last) -> bool {
         if (!wait_all(h_full_bar, static_cast<uint32_t>(t) & 1u, kStatusMma, abort_flag)) return false;
         if (first && useq > 0 && !wait_all(u_free_bar, static_cast<uint32_t>(useq - 1) & 1u, kStatusMma, abort_flag))
           return false;
+        if (!wait_all(sf_full_bar(sfb), sf_phase, kStatusMma, abort_flag)) return false;
         tc_fence_after();
         const uint32_t la = (h_tile >> 4) | (1u << 16);
-        const uint32_t lb = (slice_buf(t & 1) >> 4) | (1u << 16);
+        const uint32_t lb = lo0 + stage * (L::kStage >> 4);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t a_off = static_cast<uint32_t>((j >> 2) * (16384 >> 4) + (j & 3) * 2);
@@ -301,7 +300,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           mma_bf16_pair_warp(d_u, desc_join(la + a_off, hi_ab), desc_join(lb + b_off, hi_ab), idesc_u,
                              (first && j == 0) ? 0u : 1u);
         }
-        tc_commit_pair_mc_warp(slice_empty_bar(t & 1), kBoth);
+        tc_commit_pair_mc_warp(empty_bar(stage), kBoth);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++sfb == kSfBufs) { sfb = 0; sf_phase ^= 1u; }
         tc_commit_pair_mc_warp(h_empty_bar, kBoth);
         if (last) {
           tc_commit_pair_mc_warp(u_done_bar, kBoth);
@@ -371,55 +372,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int stage = 0, sfb = 0, slots_done = 0;
     uint32_t phase = 0;
     const int lr_slots = (r + kLrChunk - 1) / kLrChunk;
-    bool ok = true;
+    // one ring slot: wait for this CTA's data, store its scale atoms (K-step slots only), report it
+    auto slot = [&](bool has_sf) -> bool {
+      const bool got_data = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
+      if (!__all_sync(0xffffffffu, got_data)) return false;
+      uint4 fa[4], fb[4 * G::kSfAtomsB];
+      if (has_sf) {
+        const uint8_t* sfs = smem + stage * L::kStage + G::kOffSfa + lane * 16;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) fa[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
+#pragma unroll
+        for (int i = 0; i < 4 * G::kSfAtomsB; ++i)
+          fb[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + G::kOffSfb + lane * 16 + 512 * i);
+      }
+      bool got = true;
+      if (slots_done >= kSfBufs) {
+        int ps = stage - kSfBufs;
+        uint32_t pp = phase;
+        if (ps < 0) {
+          ps += STAGES;
+          pp ^= 1u;
+        }
+        got = mbar_wait_bounded(empty_bar(ps), pp, wait_ns, status, kStatusEpilogue, abort_flag);
+      }
+      if (!__all_sync(0xffffffffu, got)) return false;
+      if (has_sf) {
+        tc_fence_after();
+        const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + G::kColSf + sfb * G::kSfCols;
+        tmem_st_x16(tsf, fa);
+#pragma unroll
+        for (int h = 0; h < G::kSfAtomsB; ++h) {
+          const uint4 v[4] = {fb[4 * h], fb[4 * h + 1], fb[4 * h + 2], fb[4 * h + 3]};
+          tmem_st_x16(tsf + 16 + 16 * h, v);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_map(sf_full_bar(sfb), 0));
+      ++slots_done;
+      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      if (++sfb == kSfBufs) sfb = 0;
+      return true;
+    };
+    // per tile: its low-rank slots, its K steps, then (from the second tile on) the slot that
+    // carries the previous tile's L1s' slice; after the last tile, that tile's slice slot
+    bool ok = true, any = false;
     for (int unit = pair0; ok && unit < args.num_units; unit += npairs) {
       int m_pair, split, n_beg, n_end;
       unit_range(unit, args.splits, args.n_tiles, m_pair, split, n_beg, n_end);
       for (int n_blk = n_beg; ok && n_blk < n_end; ++n_blk) {
-        for (int slot = 0; slot < lr_slots + args.k_iters; ++slot) {
-          const bool got_data = mbar_wait_bounded(full_bar(stage), phase, wait_ns, status, kStatusEpilogue, abort_flag);
-          if (!__all_sync(0xffffffffu, got_data)) { ok = false; break; }
-          const bool has_sf = slot >= lr_slots;
-          uint4 fa[4], fb[4 * G::kSfAtomsB];
-          if (has_sf) {
-            const uint8_t* sfs = smem + stage * L::kStage + G::kOffSfa + lane * 16;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) fa[i] = *reinterpret_cast<const uint4*>(sfs + 512 * i);
-#pragma unroll
-            for (int i = 0; i < 4 * G::kSfAtomsB; ++i)
-              fb[i] = *reinterpret_cast<const uint4*>(smem + stage * L::kStage + G::kOffSfb + lane * 16 + 512 * i);
-          }
-          bool got = true;
-          if (slots_done >= kSfBufs) {
-            int ps = stage - kSfBufs;
-            uint32_t pp = phase;
-            if (ps < 0) {
-              ps += STAGES;
-              pp ^= 1u;
-            }
-            got = mbar_wait_bounded(empty_bar(ps), pp, wait_ns, status, kStatusEpilogue, abort_flag);
-          }
-          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-          if (has_sf) {
-            tc_fence_after();
-            const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + G::kColSf + sfb * G::kSfCols;
-            tmem_st_x16(tsf, fa);
-#pragma unroll
-            for (int h = 0; h < G::kSfAtomsB; ++h) {
-              const uint4 v[4] = {fb[4 * h], fb[4 * h + 1], fb[4 * h + 2], fb[4 * h + 3]};
-              tmem_st_x16(tsf + 16 + 16 * h, v);
-            }
-            tmem_wait_st();
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(cluster_map(sf_full_bar(sfb), 0));
-          ++slots_done;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++sfb == kSfBufs) sfb = 0;
-        }
+        for (int sl = 0; ok && sl < lr_slots + args.k_iters; ++sl) ok = slot(sl >= lr_slots);
+        if (ok && any) ok = slot(false);
+        any = true;
       }
     }
+    if (ok && any) slot(false);
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..9)
     // Warp (q, h): TMEM lane quadrant q = warp % 4 (rows q*32 .. q*32+31 of this CTA's 128) and
@@ -548,11 +556,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                        m_blk * 128 + q * 32);
           bulk_commit_group();
         }
-        // the tile's slice of L1s' has landed in this CTA: then both halves of the pair's U' MMA
-        // operands are ready once all 16 warps have arrived
-        const bool got_slice = mbar_wait_bounded(lf_full_bar(tseq & 1), static_cast<uint32_t>(tseq >> 1) & 1u,
-                                                 wait_ns, status, kStatusEpilogue, abort_flag);
-        if (!__all_sync(0xffffffffu, got_slice)) { ok = false; break; }
+        // both CTAs' h tiles are the U' MMA's A operand: ready once all 16 warps have arrived (the
+        // issuer waits for the slot that carries the tile's L1s' slice on its own)
         if (lane == 0) mbar_arrive_release_cluster(cluster_map(h_full_bar, 0));
         // pass 2: this row's four 16-column blocks of h, quantized for the next layer exactly as
         // kernel 1 would quantize them (rows past M get zero codes and scales, as kernel 1 writes)

@@ -10,7 +10,8 @@ model asserts that its previous user is done:
   * a slot's MMAs are issued only once both CTAs' copies of it have landed;
   * the accumulator is overwritten only after every epilogue warp has read the previous tile;
   * the h tile is rewritten only after the previous tile's U' MMAs read it;
-  * an L1s' slice buffer is refilled only after the U' MMAs two tiles back read it;
+  * a tile's L1s' slice travels in a ring slot of its own, loaded after the next tile's K steps:
+    its U' MMAs are issued only once both CTAs' halves of it have landed, and release the slot;
   * a unit's first U' MMA (accumulate = 0) comes only after the previous unit's U' was drained.
 Over many schedules and unit layouts the model must finish without a deadlock or stray arrivals,
 and every wait must pass on exactly the completion it means (a parity wait a phase early passes too
@@ -22,7 +23,7 @@ import random
 import pytest
 
 SF_BUFS = 4
-KERNEL_STAGES = 4   # the fused kernel's ring depth (kFusedStages)
+KERNEL_STAGES = 5   # the fused kernel's ring depth (kFusedStages)
 
 # Waits whose removal must break the protocol. Two of the kernel's waits are implied by others:
 #  * issuer.u_free: a unit's first U' MMA waits on h_full, and the draining warps arrive on h_full
@@ -30,8 +31,8 @@ KERNEL_STAGES = 4   # the fused kernel's ring depth (kFusedStages)
 #  * sf.release, while the ring has no more stages than scale buffers: a writer cannot see the
 #    data of the slot SF_BUFS ahead before this slot is consumed. With a deeper ring (the NVFP4
 #    GEMM runs 5 stages) it is needed, which test_every_wait_is_needed checks at 6 stages.
-WAITS = ["producer.empty", "producer.slice_empty", "issuer.acce", "issuer.sf_full", "issuer.h_full",
-         "sf.full", "sf.release", "epi.accf", "epi.u_done", "epi.h_empty", "epi.lf_full"]
+WAITS = ["producer.empty", "issuer.acce", "issuer.sf_full", "issuer.slice_sf_full", "issuer.h_full",
+         "sf.full", "sf.release", "epi.accf", "epi.u_done", "epi.h_empty"]
 
 
 class Barrier:
@@ -61,9 +62,6 @@ def run_model(units, r, k_iters, seed, skip=(), stages=KERNEL_STAGES):
             bar(f"full{c}.{s}", 1)
             bar(f"empty{c}.{s}", 1)
         bar(f"accf{c}", 1)
-        for b in range(2):
-            bar(f"lf_full{c}.{b}", 1)
-            bar(f"slice_empty{c}.{b}", 1)
         bar(f"h_empty{c}", 1)
         bar(f"u_done{c}", 1)
     bar("acce", 16)                     # 8 epilogue warps x 2 CTAs
@@ -90,22 +88,23 @@ def run_model(units, r, k_iters, seed, skip=(), stages=KERNEL_STAGES):
 
     tiles = [(t == 0, t == n - 1) for n in units for t in range(n)]
 
+    # the ring slots of one pair in order: per tile its low-rank and K-step slots, then (from the
+    # second tile on) the previous tile's slice slot; after the last tile, its slice slot
+    order = []
+    for t in range(len(tiles)):
+        order += ["data"] * slots + (["slice"] if t > 0 else [])
+    if tiles:
+        order.append("slice")
+
     def producer(c):
-        stage, tseq = 0, 0
+        stage = 0
         uses = [0] * STAGES
-        for _ in tiles:
-            for _ in range(slots):
-                yield from wait("producer.empty", f"empty{c}.{stage}", uses[stage] - 1)
-                assert done(f"empty{c}.{stage}") >= uses[stage], "ring stage refilled while its MMAs read it"
-                uses[stage] += 1
-                later(f"full{c}.{stage}")
-                stage = (stage + 1) % STAGES
-            b, use = tseq & 1, tseq >> 1
-            if use > 0:
-                yield from wait("producer.slice_empty", f"slice_empty{c}.{b}", use - 1)
-            assert done(f"slice_empty{c}.{b}") >= use, "slice buffer refilled while U' MMAs read it"
-            later(f"lf_full{c}.{b}")
-            tseq += 1
+        for _ in order:
+            yield from wait("producer.empty", f"empty{c}.{stage}", uses[stage] - 1)
+            assert done(f"empty{c}.{stage}") >= uses[stage], "ring stage refilled while its MMAs read it"
+            uses[stage] += 1
+            later(f"full{c}.{stage}")
+            stage = (stage + 1) % STAGES
 
     def issuer():
         stage, sfb, useq, g = 0, 0, 0, 0
@@ -113,20 +112,25 @@ def run_model(units, r, k_iters, seed, skip=(), stages=KERNEL_STAGES):
         pend = None
 
         def issue_u(t, first, last):
-            nonlocal useq
+            nonlocal useq, stage, sfb, g
             yield from wait("issuer.h_full", "h_full", t)
             if first and useq > 0:
                 yield from wait("issuer.u_free", "u_free", useq - 1)
+            yield from wait("issuer.slice_sf_full", f"sf_full{sfb}", sf_uses[sfb])
+            sf_uses[sfb] += 1
             for c in (0, 1):
-                assert done(f"lf_full{c}.{t & 1}") >= (t >> 1) + 1, "U' MMA before the slice landed"
+                assert done(f"full{c}.{stage}") >= g // STAGES + 1, "U' MMA before a CTA's slice landed"
             assert done("h_full") >= t + 1, "U' MMA before both h tiles were written"
             if first:
                 assert done("u_free") >= useq, "U' overwritten before the previous unit was drained"
             for c in (0, 1):
-                later(f"slice_empty{c}.{t & 1}")
+                later(f"empty{c}.{stage}")
                 later(f"h_empty{c}")
                 if last:
                     later(f"u_done{c}")
+            stage = (stage + 1) % STAGES
+            sfb = (sfb + 1) % SF_BUFS
+            g += 1
             if last:
                 useq += 1
 
@@ -156,18 +160,17 @@ def run_model(units, r, k_iters, seed, skip=(), stages=KERNEL_STAGES):
         full_uses = [0] * STAGES
         released = [0] * STAGES
         stage, sfb, n = 0, 0, 0
-        for _ in tiles:
-            for _ in range(slots):
-                yield from wait("sf.full", f"full{c}.{stage}", full_uses[stage])
-                full_uses[stage] += 1
-                if n >= SF_BUFS:
-                    ps = (stage - SF_BUFS) % STAGES               # the slot SF_BUFS back
-                    yield from wait("sf.release", f"empty{c}.{ps}", released[ps])
-                    released[ps] += 1
-                B[f"sf_full{sfb}"].arrive(4)
-                n += 1
-                stage = (stage + 1) % STAGES
-                sfb = (sfb + 1) % SF_BUFS
+        for _ in order:
+            yield from wait("sf.full", f"full{c}.{stage}", full_uses[stage])
+            full_uses[stage] += 1
+            if n >= SF_BUFS:
+                ps = (stage - SF_BUFS) % STAGES               # the slot SF_BUFS back
+                yield from wait("sf.release", f"empty{c}.{ps}", released[ps])
+                released[ps] += 1
+            B[f"sf_full{sfb}"].arrive(4)
+            n += 1
+            stage = (stage + 1) % STAGES
+            sfb = (sfb + 1) % SF_BUFS
 
     def epilogue(c, drains):
         useq = 0
@@ -186,7 +189,6 @@ def run_model(units, r, k_iters, seed, skip=(), stages=KERNEL_STAGES):
                 yield from wait("epi.h_empty", f"h_empty{c}", tseq - 1)
             assert done(f"h_empty{c}") >= tseq, "h tile rewritten while U' MMAs read it"
             B["acce"].arrive()
-            yield from wait("epi.lf_full", f"lf_full{c}.{tseq & 1}", tseq >> 1)
             B["h_full"].arrive()
             if last:
                 useq += 1
