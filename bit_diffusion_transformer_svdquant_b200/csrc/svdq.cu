@@ -49,7 +49,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct DeviceState {
   bool ready = false;
   int sm_count = 0;
-  int max_pairs[3] = {0, 0, 0};  // co-resident CTA pairs of the GEMM kernel for n_tile 256, 192, 128
+  int max_pairs[4] = {0, 0, 0, 0};  // co-resident CTA pairs of the GEMM kernel for n_tile 256, 192, 128, 384
   int k1_clusters[4][4] = {};     // co-resident kernel-1 clusters, by r (0/16/32/64) and size - 1 (1..4)
   svdq_status status = SVDQ_OK;
   std::string error;
@@ -60,6 +60,7 @@ DeviceState g_dev[64];
 constexpr int kStagesTile256 = 5;
 constexpr int kStagesTile192 = 5;
 constexpr int kStagesTile128 = 6;
+constexpr int kStagesTile384 = 4;
 
 using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -97,6 +98,9 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 128, kStagesTile128>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::GemmLayout<128, kStagesTile128>::kSmem));
+    SVDQ_CUDA(cudaFuncSetAttribute(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 384, kStagesTile384>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   svdq::GemmLayout<384, kStagesTile384>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<0, svdq::Nvfp4Act>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    svdq::Q1Layout<0>::kSmem));
     SVDQ_CUDA(cudaFuncSetAttribute(svdq::quant_act_kernel<16, svdq::Nvfp4Act>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -128,6 +132,10 @@ svdq_status device_ready(int* dev_out, int* sm_out) {
       return s;
     if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 128, kStagesTile128>),
                                   svdq::GemmLayout<128, kStagesTile128>::kSmem, &st.max_pairs[2]);
+        s != SVDQ_OK)
+      return s;
+    if (svdq_status s = max_pairs(reinterpret_cast<const void*>(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 384, kStagesTile384>),
+                                  svdq::GemmLayout<384, kStagesTile384>::kSmem, &st.max_pairs[3]);
         s != SVDQ_OK)
       return s;
     // how many kernel-1 clusters of 1, 2, 3 and 4 CTAs (one CTA per SM) can be resident at once
@@ -193,18 +201,31 @@ CUtensorMapSwizzle lr_swizzle(int r) { return r == 16 ? CU_TENSOR_MAP_SWIZZLE_32
 
 bool valid_r(int r) { return r == 0 || r == 16 || r == 32 || r == 64; }
 
-// GEMM tile width along N: 256 where it divides N (the widest MMA: fewest bytes streamed per
-// flop), else 192, else 128. SVDQ_N_TILE overrides it with another valid width.
-int choose_n_tile(int N) {
+// The 384-wide NVFP4 tile (two pair MMAs per K chunk): a weight without the SwiGLU interleave whose
+// N is a multiple of 768, so that its blob has the same size as at 256 (N / 128 scale atoms per K
+// atom either way) and svdq_weight_bytes need not know whether a weight is SwiGLU.
+bool wide_tile_ok(int N, int swiglu) { return !swiglu && N % 768 == 0; }
+
+// GEMM tile width along N: the widest that divides N, for the fewest operand bytes streamed per
+// flop: 384 (where wide_tile_ok and `wide`: the NVFP4 GEMM), else 256, 192, 128. SVDQ_N_TILE
+// overrides it with another valid width.
+int choose_n_tile(int N, int swiglu, bool wide) {
   const char* env = getenv("SVDQ_N_TILE");
   if (env != nullptr) {
     const int t = atoi(env);
     if ((t == 256 || t == 192 || t == 128) && N % t == 0) return t;
+    if (t == 384 && wide && wide_tile_ok(N, swiglu)) return t;
   }
+  if (wide && wide_tile_ok(N, swiglu)) return 384;
   if (N % 256 == 0) return 256;
   if (N % 192 == 0) return 192;
   if (N % 128 == 0) return 128;
   return 0;
+}
+// A GEMM tile width a descriptor of an NVFP4 weight may hold.
+bool valid_n_tile(int N, int n_tile, int swiglu) {
+  if (n_tile == 384) return wide_tile_ok(N, swiglu);
+  return (n_tile == 256 || n_tile == 192 || n_tile == 128) && N % n_tile == 0;
 }
 
 struct WeightLayout {
@@ -250,14 +271,15 @@ ActLayout act_layout(int M, int K, int r) {
 }
 
 bool shape_ok(int N, int K, int r) {
-  return N > 0 && K > 0 && K % 256 == 0 && valid_r(r) && K <= (1 << 20) && N <= (1 << 20) && choose_n_tile(N) > 0;
+  return N > 0 && K > 0 && K % 256 == 0 && valid_r(r) && K <= (1 << 20) && N <= (1 << 20) &&
+         choose_n_tile(N, 0, false) > 0;
 }
 
 // The descriptors are plain structs that a caller may also fill by hand: before a launch reads
 // through them, check that they describe a layout that svdq_pack_weight / svdq_act_bind can produce.
 svdq_status check_weight(const svdq_weight* w) {
   const int t = w->n_tile;
-  if ((t != 256 && t != 192 && t != 128) || w->N <= 0 || w->N % t != 0 || w->N > (1 << 20) || w->K <= 0 ||
+  if (w->N <= 0 || !valid_n_tile(w->N, t, w->swiglu_interleaved) || w->N > (1 << 20) || w->K <= 0 ||
       w->K % 256 != 0 || w->K > (1 << 20) || !valid_r(w->r))
     return fail(SVDQ_ERR_INVALID_ARG, "weight descriptor N=%d K=%d r=%d n_tile=%d is not one svdq_pack_weight makes",
                 w->N, w->K, w->r, t);
@@ -373,12 +395,12 @@ const char* svdq_last_error(void) { return g_last_error.c_str(); }
 
 size_t svdq_weight_bytes(int N, int K, int r) {
   if (!shape_ok(N, K, r)) return 0;
-  return weight_layout(N, K, r, choose_n_tile(N)).total;
+  return weight_layout(N, K, r, choose_n_tile(N, 0, true)).total;
 }
 
 size_t svdq_weight_bytes_tiled(int N, int K, int r, int n_tile) {
   if (N <= 0 || K <= 0 || K % 256 != 0 || K > (1 << 20) || N > (1 << 20) || !valid_r(r) ||
-      (n_tile != 256 && n_tile != 192 && n_tile != 128) || N % n_tile != 0)
+      !valid_n_tile(N, n_tile, 0))
     return 0;
   return weight_layout(N, K, r, n_tile).total;
 }
@@ -424,7 +446,7 @@ svdq_status svdq_pack_weight(const float* R_nk, const uint16_t* L1s_kr, const ui
   if (!aligned16(R_nk) || !aligned16(inv_lambda) || (r > 0 && (!aligned16(L1s_kr) || !aligned16(L2_rn))))
     return fail(SVDQ_ERR_UNSUPPORTED, "inputs must be 16-byte aligned");
   if (reinterpret_cast<uintptr_t>(dst) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "dst not 256-byte aligned");
-  const int n_tile = choose_n_tile(N);
+  const int n_tile = choose_n_tile(N, swiglu, true);
   const WeightLayout l = weight_layout(N, K, r, n_tile);
   if (dst_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "weight buffer %zu bytes < %zu", dst_bytes, l.total);
   int dev, sms;
@@ -463,8 +485,9 @@ svdq_status svdq_weight_bind(int N, int K, int r, int swiglu, int n_tile, void* 
                              svdq_weight* out) {
   if (out == nullptr || blob == nullptr) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
   if (N <= 0 || K <= 0 || K % 256 != 0 || K > (1 << 20) || N > (1 << 20) || !valid_r(r) ||
-      (n_tile != 256 && n_tile != 192 && n_tile != 128) || N % n_tile != 0)
-    return fail(SVDQ_ERR_UNSUPPORTED, "weight shape N=%d K=%d r=%d n_tile=%d unsupported", N, K, r, n_tile);
+      !valid_n_tile(N, n_tile, swiglu))
+    return fail(SVDQ_ERR_UNSUPPORTED, "weight shape N=%d K=%d r=%d n_tile=%d swiglu=%d unsupported", N, K, r, n_tile,
+                swiglu);
   if (reinterpret_cast<uintptr_t>(blob) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "blob not 256-byte aligned");
   const WeightLayout l = weight_layout(N, K, r, n_tile);
   if (blob_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "weight blob %zu bytes < %zu", blob_bytes, l.total);
@@ -654,12 +677,15 @@ svdq_status svdq_gemm(const svdq_act* act, const svdq_weight* w, const uint16_t*
   int max_pairs = 0;
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    max_pairs = g_dev[dev].max_pairs[n_tile == 256 ? 0 : n_tile == 192 ? 1 : 2];
+    max_pairs = g_dev[dev].max_pairs[n_tile == 256 ? 0 : n_tile == 192 ? 1 : n_tile == 128 ? 2 : 3];
   }
   const int pairs = g.num_tiles < max_pairs ? g.num_tiles : max_pairs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (n_tile == 256)
+  if (n_tile == 384)
+    e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 384, kStagesTile384>, 2 * pairs,
+                         svdq::GemmLayout<384, kStagesTile384>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
+  else if (n_tile == 256)
     e = launch_pair_gemm(svdq::pair_gemm_kernel<svdq::Nvfp4Gemm, 256, kStagesTile256>, 2 * pairs,
                          svdq::GemmLayout<256, kStagesTile256>::kSmem, st, tmA, tmB, tmU, tmL2, tmY, g);
   else if (n_tile == 192)
@@ -894,7 +920,7 @@ svdq_status svdq_fp8r_pack_weight(const float* R_nk, const uint16_t* L1s_kr, con
   if (!aligned16(R_nk) || !aligned16(inv_lambda) || (r > 0 && (!aligned16(L1s_kr) || !aligned16(L2_rn))))
     return fail(SVDQ_ERR_UNSUPPORTED, "inputs must be 16-byte aligned");
   if (reinterpret_cast<uintptr_t>(dst) % kAlign) return fail(SVDQ_ERR_UNSUPPORTED, "dst not 256-byte aligned");
-  const int n_tile = choose_n_tile(N);
+  const int n_tile = choose_n_tile(N, swiglu, false);
   const Fp8rWeightLayout l = fp8r_weight_layout(N, K, r);
   if (dst_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "FP8 weight buffer %zu bytes < %zu", dst_bytes, l.total);
   int dev, sms;

@@ -230,14 +230,15 @@ struct Fp8Gemm {
   using Args = GemmArgs;
   static constexpr bool kScales = false;
   static constexpr bool kL2HiLo = true;
-  __device__ static constexpr uint32_t idesc(int m, int n) { return idesc_e4m3(m, n); }
-  template <int SF_ATOMS_B>
-  __device__ static void kstep(uint32_t d, uint32_t la, uint32_t lb, uint32_t hi_ab, uint32_t idesc_k, uint32_t,
-                               uint32_t accumulate) {
-    mma_e4m3_pair_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_k, accumulate);
-    mma_e4m3_pair_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_k, 1u);
-    mma_e4m3_pair_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_k, 1u);
-    mma_e4m3_pair_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_k, 1u);
+  // the four MMAs of a 128-element K step (each K = 32, 32 bytes of codes per row)
+  template <int N_TILE, int SF_ATOMS_B>
+  __device__ static void kstep(uint32_t d, uint32_t la, uint32_t lb, uint32_t hi_ab, uint32_t, uint32_t accumulate) {
+    static_assert(N_TILE <= 256, "FP8 tiles are at most 256 wide");
+    constexpr uint32_t id = idesc_e4m3(256, N_TILE);
+    mma_e4m3_pair_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), id, accumulate);
+    mma_e4m3_pair_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), id, 1u);
+    mma_e4m3_pair_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), id, 1u);
+    mma_e4m3_pair_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), id, 1u);
   }
   struct Epi {
     float sx;

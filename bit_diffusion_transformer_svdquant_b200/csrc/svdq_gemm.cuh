@@ -32,11 +32,14 @@
 //                shape, so copying 12 atoms per K step with tcgen05.cp starved the MMAs; stores
 //                from four warps run beside the MMAs without slowing them.
 // TMEM (512 columns): the accumulator (n_tile columns; two buffers when n_tile = 128) and 4 scale
-// buffers of 16 + 16 * ceil(n_tile / 128) columns. Measured on B200: with only 2 scale buffers
-// the commit -> writer -> remote arrive -> issuer round trip (~900 cycles across the pair) could
-// not hide under one K step; and one CTA per 128 x 192 tile had to stream 48 KB per 384-cycle K
-// step from L2 per SM, above what a B200 SM sustained in isolation (~75-90 B per cycle), against
-// 38 KB per 512 cycles here.
+// buffers of 16 + 16 * ceil(n_tile / 128) columns (2 beside the 384-column accumulator). Measured
+// on B200: with only 2 scale buffers the commit -> writer -> remote arrive -> issuer round trip
+// (~900 cycles across the pair) could not hide under a 256-wide K step; and one CTA per 128 x 192
+// tile had to stream 48 KB per 384-cycle K step from L2 per SM, above what a B200 SM sustained in
+// isolation (~75-90 B per cycle), against 38 KB per 512 cycles here.
+// The 384-wide tile (4-stage ring) issues each K chunk as two MMAs, N = 256 and N = 128, on the
+// same A: 48 KB per CTA per 768-cycle K step, 16 % fewer operand bytes per flop than at 256, for a
+// kernel whose time follows the bytes it streams from L2.
 // Every mbarrier wait is bounded (global timer); a wait that runs out records a status bit, sets
 // a shared abort flag so that the other roles of the CTA stop too, and the kernel drains its own
 // copies and MMAs before the cluster-wide barrier that precedes freeing TMEM.
@@ -80,8 +83,9 @@ struct PairGemmLayout {
   // a format whose L2^T is kept as a bf16 hi/lo pair, its lo half (kOffL2Lo)
   static constexpr int kOffL2Lo = kOffB + kBRows * 32 * 2;
   // TMEM scale-factor buffer (one K step): SFA 4 MMAs x 4 columns, then SFB 4 MMAs x 4 x atoms.
+  // Four buffers beside an accumulator of up to 256 columns; two beside the 384-column one.
   static constexpr int kSfCols = SCALES ? 16 + 16 * kSfAtomsB : 0;
-  static constexpr int kSfBufs = SCALES ? 4 : 0;
+  static constexpr int kSfBufs = SCALES ? (N_TILE > 256 ? 2 : 4) : 0;
   static constexpr int kAccBufs = (2 * N_TILE + kSfBufs * kSfCols <= 512) ? 2 : 1;
   static constexpr int kColSf = kAccBufs * N_TILE;  // kSfBufs buffers of kSfCols columns from here
   // epilogue staging: 8 warps x 4 KB (two 32 x 32 bf16 boxes or one fp32 box in flight)
@@ -97,6 +101,7 @@ struct PairGemmLayout {
   static_assert(kColSf + kSfBufs * kSfCols <= 512, "TMEM budget");
   static_assert(kSfBufs <= STAGES, "a scale buffer's previous slot must still own its ring stage");
   static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(N_TILE <= 256 || (SCALES && N_TILE == 384), "the 384-wide tile is an NVFP4 tile");
 };
 template <int N_TILE, int STAGES>
 using GemmLayout = PairGemmLayout<true, N_TILE, STAGES>;
@@ -135,18 +140,33 @@ struct Nvfp4Gemm {
   using Args = GemmArgs;
   static constexpr bool kScales = true;
   static constexpr bool kL2HiLo = false;
-  __device__ static constexpr uint32_t idesc(int m, int n) { return idesc_nvfp4(m, n); }
-  // the four MMAs of a 256-element K step (each K = 64, 32 bytes of codes per row)
-  template <int SF_ATOMS_B>
-  __device__ static void kstep(uint32_t d, uint32_t la, uint32_t lb, uint32_t hi_ab, uint32_t idesc_k,
-                               uint32_t tsf, uint32_t accumulate) {
-    mma_nvfp4_pair_warp(d, desc_join(la, hi_ab), desc_join(lb, hi_ab), idesc_k, tsf, tsf + 16, accumulate);
-    mma_nvfp4_pair_warp(d, desc_join(la + 2u, hi_ab), desc_join(lb + 2u, hi_ab), idesc_k, tsf + 4,
-                        tsf + 16 + 4 * SF_ATOMS_B, 1u);
-    mma_nvfp4_pair_warp(d, desc_join(la + 4u, hi_ab), desc_join(lb + 4u, hi_ab), idesc_k, tsf + 8,
-                        tsf + 16 + 8 * SF_ATOMS_B, 1u);
-    mma_nvfp4_pair_warp(d, desc_join(la + 6u, hi_ab), desc_join(lb + 6u, hi_ab), idesc_k, tsf + 12,
-                        tsf + 16 + 12 * SF_ATOMS_B, 1u);
+  // the MMAs of a 256-element K step: four of K = 64 (32 bytes of codes per row); the SFA of MMA j
+  // at tsf + 4j, its SFB atoms (128 tile columns each) from tsf + 16 + 4 SF_ATOMS_B j on
+  template <int N_TILE, int SF_ATOMS_B>
+  __device__ static void kstep(uint32_t d, uint32_t la, uint32_t lb, uint32_t hi_ab, uint32_t tsf,
+                               uint32_t accumulate) {
+    if constexpr (N_TILE <= 256) {
+      constexpr uint32_t id = idesc_nvfp4(256, N_TILE);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        mma_nvfp4_pair_warp(d, desc_join(la + 2u * j, hi_ab), desc_join(lb + 2u * j, hi_ab), id, tsf + 4 * j,
+                            tsf + 16 + 4 * SF_ATOMS_B * j, j == 0 ? accumulate : 1u);
+    } else {
+      // 384 columns as N = 256 (accumulator columns 0..255; the first 128 rows of each CTA's B box,
+      // SFB atoms 3j and 3j + 1) and N = 128 (columns 256..383; the box's last 64 rows, 16 KB on,
+      // SFB atom 3j + 2), both on the same A
+      constexpr uint32_t id_a = idesc_nvfp4(256, 256), id_b = idesc_nvfp4(256, N_TILE - 256);
+      constexpr uint32_t kB2 = (128 * 128) >> 4;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t a = desc_join(la + 2u * j, hi_ab);
+        const uint32_t acc = j == 0 ? accumulate : 1u;
+        mma_nvfp4_pair_warp(d, a, desc_join(lb + 2u * j, hi_ab), id_a, tsf + 4 * j, tsf + 16 + 4 * SF_ATOMS_B * j,
+                            acc);
+        mma_nvfp4_pair_warp(d + 256, a, desc_join(lb + kB2 + 2u * j, hi_ab), id_b, tsf + 4 * j,
+                            tsf + 16 + 4 * SF_ATOMS_B * j + 8, acc);
+      }
+    }
   }
   // per tile row: y = alpha acc (+ bias) for 8 accumulator columns g0.. (GEMM order) of v[off..]
   struct Epi {
@@ -344,8 +364,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int num_tiles = args.num_tiles, k_iters = args.k_iters;
       const int rc = r < kLrChunk ? r : kLrChunk;
       const int nj = rc >> 4;
-      const uint32_t idesc_k = F::idesc(256, N_TILE);
-      const uint32_t idesc_lr = idesc_bf16(256, N_TILE);
+      // the low-rank MMAs span the tile like the K steps: one of N = n_tile, or 256 + 128 columns
+      constexpr int kLrN = N_TILE <= 256 ? N_TILE : 256;
+      const uint32_t idesc_lr = idesc_bf16(256, kLrN);
+      const uint32_t idesc_lr2 = idesc_bf16(256, N_TILE > 256 ? N_TILE - 256 : 16);
       // descriptor halves: low = start address / 16 | LBO (16 B) / 16 << 16; high = SBO / 16 |
       // version 1 | swizzle mode << 29
       const uint32_t lo0 = (sbase >> 4) | (1u << 16);
@@ -377,6 +399,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint64_t u_lo = desc_join(lo + (kOffULo >> 4) + 2u * j, hi_lr);
             const uint64_t l_hi = desc_join(lo + (L::kOffB >> 4) + 2u * j, hi_lr);
             mma_bf16_pair_warp(d, u_hi, l_hi, idesc_lr, accumulate);
+            if constexpr (N_TILE > 256) {
+              // columns 256..383: the last 64 rows of each CTA's L2^T box
+              const uint64_t l_hi2 = desc_join(lo + ((L::kOffB + 128 * rc * 2) >> 4) + 2u * j, hi_lr);
+              mma_bf16_pair_warp(d + 256, u_hi, l_hi2, idesc_lr2, accumulate);
+              mma_bf16_pair_warp(d + 256, u_lo, l_hi2, idesc_lr2, 1u);
+            }
             mma_bf16_pair_warp(d, u_lo, l_hi, idesc_lr, 1u);
             if constexpr (F::kL2HiLo)
               mma_bf16_pair_warp(d, u_hi, desc_join(lo + (L::kOffL2Lo >> 4) + 2u * j, hi_lr), idesc_lr, 1u);
@@ -391,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t la = lo0 + stage * (L::kStage >> 4);
           const uint32_t lb = la + (L::kOffB >> 4);
-          F::template kstep<L::kSfAtomsB>(d, la, lb, hi_ab, idesc_k, tsf0 + sfb * L::kSfCols, accumulate);
+          F::template kstep<N_TILE, L::kSfAtomsB>(d, la, lb, hi_ab, tsf0 + sfb * L::kSfCols, accumulate);
           accumulate = 1;
           tc_commit_pair_mc_warp(empty_bar(stage), kBoth);
           next_slot();
@@ -572,21 +600,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // the two staging boxes, later chunks stay packed in registers; the accumulator is released
         // after the last round's loads and only then are the boxes stored (measured on B200:
         // staging and storing each chunk before the next load took ~700 cycles per chunk, all of it
-        // on the issuer's path to the next tile)
+        // on the issuer's path to the next tile). The 384-wide tile's six chunks per warp load their
+        // last two rounds one chunk at a time, which keeps the packed chunks and the loaded ones
+        // within the register budget.
         const int c_beg = h * kPlainPerWarp;
-        uint32_t pk[2][16];
+        uint32_t pk[kPlainPerWarp > 2 ? kPlainPerWarp - 2 : 1][16];
         boxes_free();
 #pragma unroll
-        for (int i = 0; i < kPlainPerWarp; i += 2) {
+        for (int i = 0; i < kPlainPerWarp; i += (kPlainPerWarp > 4 && i >= 4) ? 1 : 2) {
+          const bool pair = !(kPlainPerWarp > 4 && i >= 4) && i + 1 < kPlainPerWarp;
           float v[2][32];
           tmem_ld_32x32(tb + (c_beg + i) * 32, v[0]);
-          if (i + 1 < kPlainPerWarp) tmem_ld_32x32(tb + (c_beg + i + 1) * 32, v[1]);
+          if (pair) tmem_ld_32x32(tb + (c_beg + i + 1) * 32, v[1]);
           tmem_wait_ld();
-          if (i + 2 >= kPlainPerWarp) release_acc();
+          if (i + (pair ? 2 : 1) >= kPlainPerWarp) release_acc();
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int j = i + u;
-            if (j < kPlainPerWarp) {
+            if (j < kPlainPerWarp && (u == 0 || pair)) {
               const int g0 = n_blk * N_TILE + (c_beg + j) * 32;
               affine(ep, v[u], g0, g0);
               if (j < 2) {
@@ -622,10 +653,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           affine(ep, v, g0, g0);
           emit_f32(v, row0, g0);
         }
-      } else {
-        // SwiGLU: output chunk c pairs gate columns c*32.. with up columns n_tile/2 + c*32.. (at
-        // most two chunks per warp, one staging box each); gate GEMM column g, output (and gate
-        // bias) column j, up bias column hN + j
+      } else if constexpr (N_TILE <= 256) {
+        // SwiGLU (tiles up to 256 wide; the host packs SwiGLU weights no wider): output chunk c
+        // pairs gate columns c*32.. with up columns n_tile/2 + c*32.. (at most two chunks per warp,
+        // one staging box each); gate GEMM column g, output (and gate bias) column j, up bias
+        // column hN + j
         constexpr int kHalf = N_TILE / 2;
         const int n_mine = glu_end - glu_beg;
         if (!f32) {

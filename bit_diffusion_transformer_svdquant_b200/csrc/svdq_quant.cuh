@@ -33,25 +33,52 @@ __host__ __device__ __forceinline__ size_t act_sf_offset(int m, int kb, int K) {
   return ((static_cast<size_t>(m >> 7) * (K >> 6) + (kb >> 2)) << 9) + ((m & 31) << 4) + (((m >> 5) & 3) << 2) +
          (kb & 3);
 }
-// Same for a weight row p in GEMM order: per n_tile, per 64-wide K atom, ceil(n_tile/128) atoms.
+// A 384-wide tile runs as two pair MMAs: N = 256 over tile columns 0..255 and N = 128 over
+// 256..383, each taking half of its B rows from each CTA of the pair. Each CTA stages its share as
+// one contiguous box of 192 rows, so CTA c holds tile columns [128c, 128c + 128) followed by
+// [256 + 64c, 256 + 64c + 64). Packed (storage) row q of a tile -> tile column (the MMA's N index,
+// which is also the accumulator column) and back; the identity for the narrower tiles.
+__host__ __device__ __forceinline__ int tile_col_of_packed(int q, int n_tile) {
+  if (n_tile != 384) return q;
+  const int c = q >= 192 ? 1 : 0, s = q - 192 * c;
+  return s < 128 ? 128 * c + s : 256 + 64 * c + (s - 128);
+}
+__host__ __device__ __forceinline__ int packed_of_tile_col(int t, int n_tile) {
+  if (n_tile != 384) return t;
+  if (t < 256) return 192 * (t >> 7) + (t & 127);
+  const int u = t - 256;
+  return 192 * (u >> 6) + 128 + (u & 63);
+}
+// Same for a packed weight row p: per n_tile, per 64-wide K atom, ceil(n_tile/128) atoms of 128
+// tile columns each (the B scale layout the MMAs read from TMEM).
 __host__ __device__ __forceinline__ size_t wgt_sf_offset(int p, int kb, int K, int n_tile) {
   const int atoms = (n_tile + 127) >> 7;
-  const int nb = p / n_tile, pl = p - nb * n_tile;
+  const int nb = p / n_tile, pl = tile_col_of_packed(p - nb * n_tile, n_tile);
   const int a = pl >> 7, pr = pl & 127;
   return (((static_cast<size_t>(nb) * (K >> 6) + (kb >> 2)) * atoms + a) << 9) + ((pr & 31) << 4) +
          ((pr >> 5) << 2) + (kb & 3);
 }
-// GEMM row of original weight row n (gate/up interleave per n_tile for SwiGLU) and its inverse.
+// Packed (GEMM) row of original weight row n and its inverse: the gate/up interleave per n_tile for
+// SwiGLU (tile column t < n_tile/2 a gate row, the rest the matching up rows), then the placement of
+// tile columns in the CTAs' B boxes above.
 __host__ __device__ __forceinline__ int gemm_row_of(int n, int N, int n_tile, int swiglu) {
-  if (!swiglu) return n;
-  const int half = n_tile >> 1, hN = N >> 1;
-  if (n < hN) return (n / half) * n_tile + n % half;
-  const int u = n - hN;
-  return (u / half) * n_tile + half + u % half;
+  int g = n;
+  if (swiglu) {
+    const int half = n_tile >> 1, hN = N >> 1;
+    if (n < hN) {
+      g = (n / half) * n_tile + n % half;
+    } else {
+      const int u = n - hN;
+      g = (u / half) * n_tile + half + u % half;
+    }
+  }
+  const int nb = g / n_tile;
+  return nb * n_tile + packed_of_tile_col(g - nb * n_tile, n_tile);
 }
 __host__ __device__ __forceinline__ int orig_row_of(int p, int N, int n_tile, int swiglu) {
-  if (!swiglu) return p;
-  const int half = n_tile >> 1, nb = p / n_tile, pl = p - nb * n_tile;
+  const int nb = p / n_tile, pl = tile_col_of_packed(p - nb * n_tile, n_tile);
+  if (!swiglu) return nb * n_tile + pl;
+  const int half = n_tile >> 1;
   return pl < half ? nb * half + pl : (N >> 1) + nb * half + (pl - half);
 }
 

@@ -34,8 +34,9 @@
  *   - The per-call kernels are launched with programmatic stream serialization: one may start its
  *     set-up (barriers, tensor memory) while the kernel before it on the stream is finishing, but
  *     it reads or writes no global memory until that kernel has completed. Stream order is kept.
- *   - Shapes: K % 256 == 0; N % n_tile == 0 for the n_tile chosen at pack time (256 where it
- *     divides N, else 192, else 128; SwiGLU needs N even); r in {0, 16, 32, 64}; 1 <= M < 2^24.
+ *   - Shapes: K % 256 == 0; N % n_tile == 0 for the n_tile chosen at pack time (384 for a weight
+ *     without SwiGLU where 768 divides N, else 256 where it divides N, else 192, else 128; SwiGLU
+ *     needs N even); r in {0, 16, 32, 64}; 1 <= M < 2^24.
  *     Device pointers 16-byte aligned.
  *     Other shapes return SVDQ_ERR_UNSUPPORTED.
  *   - A device that is not sm_100 returns SVDQ_ERR_UNSUPPORTED. There is no CPU fallback.
@@ -114,9 +115,10 @@ typedef struct svdq_act {
 /* Bytes of device memory a packed weight / a quantized activation needs (0 on bad shapes). */
 SVDQ_API size_t svdq_weight_bytes(int N, int K, int r);
 SVDQ_API size_t svdq_act_bytes(int M, int K, int r);
-/* Bytes of a packed weight blob for an explicit GEMM tile width n_tile (256, 192 or 128; the
+/* Bytes of a packed weight blob for an explicit GEMM tile width n_tile (384, 256, 192 or 128; the
  * value a descriptor's n_tile field holds), e.g. to check a checkpoint's blob before re-binding it
- * with svdq_weight_bind. 0 on bad shapes or a tile width that does not divide N. */
+ * with svdq_weight_bind. 0 on bad shapes or a tile width that does not divide N (384: 768 must
+ * divide N). svdq_weight_bind also refuses n_tile 384 for a SwiGLU weight. */
 SVDQ_API size_t svdq_weight_bytes_tiled(int N, int K, int r, int n_tile);
 
 /* Offline pack of one layer's weight (not on the per-step path).
@@ -197,7 +199,7 @@ SVDQ_API svdq_status svdq_set_wait_limit_ns(unsigned long long ns);
 typedef struct svdq_fp8r_weight {
   int N, K, r;
   int swiglu_interleaved; /* 1: gate/up rows interleaved per n_tile, as for svdq_weight         */
-  int n_tile;             /* GEMM tile width along N (256 / 192 / 128, as for svdq_weight)      */
+  int n_tile;             /* GEMM tile width along N (256 / 192 / 128: the FP8 GEMM has no 384) */
   int reserved0;
   void* codes;            /* uint8 [N][K] E4M3 codes, rows in GEMM order                         */
   float* row_scale;       /* device fp32 [N] s_w per GEMM row                                    */

@@ -74,7 +74,8 @@ def _fake_pair(L):
     return w, act
 
 
-@pytest.mark.parametrize("field,value", [("n_tile", 100), ("n_tile", 0), ("N", 640), ("K", 500), ("r", 24),
+@pytest.mark.parametrize("field,value", [("n_tile", 100), ("n_tile", 0), ("n_tile", 384), ("N", 640), ("K", 500),
+                                         ("r", 24),
                                          ("codes", None), ("L2_t", None), ("M_pad", 256), ("M", 0),
                                          ("alpha", None), ("U", None)])
 def test_descriptor_checks_before_any_cuda_call(L, field, value):
@@ -153,7 +154,9 @@ def _weight_bytes_for_tile(N, K, r, n_tile):
 
 @pytest.mark.parametrize("N,tile", [(512, 256), (9216, 256), (384, 192), (1152, 192), (640, 128), (128, 128)])
 def test_tile_width_choice(L, N, tile):
-    """256 where it divides N, else 192, else 128: visible in the scale-atom count of the blob."""
+    """256 where it divides N, else 192, else 128: visible in the scale-atom count of the blob. (Where
+    768 divides N a weight without SwiGLU is packed 384 wide, whose blob has the size of the 256-wide
+    one, so the size query need not know whether the weight is SwiGLU.)"""
     K, r = 512, 32
     got = L.svdq_weight_bytes(N, K, r)
     assert got == _weight_bytes_for_tile(N, K, r, tile)
@@ -455,7 +458,8 @@ def test_weight_bind_checks(L):
 
 
 @pytest.mark.parametrize("N,K,r,tile", [(768, 512, 32, 128), (768, 512, 32, 192), (768, 512, 32, 256),
-                                        (9216, 3072, 32, 256), (384, 256, 0, 192), (640, 1024, 64, 128)])
+                                        (9216, 3072, 32, 256), (384, 256, 0, 192), (640, 1024, 64, 128),
+                                        (9216, 3072, 32, 384), (768, 256, 16, 384)])
 def test_weight_bytes_tiled(L, N, K, r, tile):
     """The size query with an explicit tile width gives the layout of that width."""
     assert L.svdq_weight_bytes_tiled(N, K, r, tile) == _weight_bytes_for_tile(N, K, r, tile)
@@ -466,6 +470,21 @@ def test_weight_bytes_tiled_rejects(L):
     assert L.svdq_weight_bytes_tiled(640, 512, 32, 256) == 0      # 256 does not divide 640
     assert L.svdq_weight_bytes_tiled(768, 500, 32, 128) == 0      # K % 256
     assert L.svdq_weight_bytes_tiled(768, 512, 24, 128) == 0      # rank
+    assert L.svdq_weight_bytes_tiled(1152, 512, 32, 384) == 0     # 384-wide needs 768 | N
+    assert L.svdq_weight_bytes_tiled(384, 512, 32, 384) == 0
+
+
+def test_wide_tile_only_without_swiglu(L):
+    """The 384-wide tile: a blob of the 256-wide size, refused for a SwiGLU weight on re-bind."""
+    import torch
+    assert L.svdq_weight_bytes_tiled(9216, 3072, 32, 384) == L.svdq_weight_bytes_tiled(9216, 3072, 32, 256)
+    w = _lib.SvdqWeight()
+    p = ctypes.c_void_p(1 << 40)
+    need = _weight_bytes_for_tile(768, 512, 32, 384)
+    assert L.svdq_weight_bind(768, 512, 32, 1, 384, p, need, ctypes.byref(w)) == 2           # SwiGLU at 384
+    assert L.svdq_weight_bind(1152, 512, 32, 0, 384, p, need, ctypes.byref(w)) == 2          # 768 does not divide N
+    if not torch.cuda.is_available():
+        assert L.svdq_weight_bind(768, 512, 32, 0, 384, p, need, ctypes.byref(w)) == 3
 
 
 def test_from_state_checks_the_blob(L):

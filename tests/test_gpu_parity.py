@@ -64,7 +64,8 @@ def test_codec_edges_through_kernel1(cuda_device):
 
 
 SMALL_CASES = [
-    # M, K, N, r, bias, swiglu     (tile width: 256 where it divides N, else 192, else 128)
+    # M, K, N, r, bias, swiglu     (tile width: 384 without SwiGLU where 768 divides N, else 256
+    # where it divides N, else 192, else 128)
     (300, 768, 384, 32, True, False),   # ragged M (odd number of 128-row blocks), two 192-wide tiles
     (1, 256, 128, 0, False, False),     # one row, no low-rank branch, 128-wide tile
     (200, 512, 768, 64, True, True),    # SwiGLU with bias, r = 64, three 256-wide tiles
@@ -74,6 +75,10 @@ SMALL_CASES = [
     (257, 512, 640, 32, True, True),    # SwiGLU on 128-wide tiles (double-buffered accumulators)
     (600, 768, 1024, 32, True, False),  # four 256-wide tiles, ragged M
     (170, 512, 384, 32, True, True),    # SwiGLU on 192-wide tiles (2 + 1 output chunks per quadrant)
+    (300, 768, 768, 32, True, False),   # 384-wide tiles (two MMAs per K chunk), ragged M
+    (1, 256, 768, 0, False, False),     # 384-wide, one row, no low-rank branch
+    (130, 1024, 768, 16, False, False), # 384-wide, r = 16 (32-byte low-rank rows)
+    (513, 256, 1536, 64, True, False),  # 384-wide, r = 64 (two low-rank slots), a ragged fifth m-tile
 ]
 
 
@@ -81,6 +86,8 @@ SMALL_CASES = [
 def test_small_shapes(cuda_device, M, K, N, r, bias, swiglu):
     X, W, b = _rand_layer(M, K, N, r, seed=M * 7 + N, bias=bias)
     c = Case(X, W, b, r, swiglu, cuda_device)
+    assert c.w.n_tile == (384 if not swiglu and N % 768 == 0 else 256 if N % 256 == 0 else 192 if N % 192 == 0
+                          else 128)
     c.check_scales()
     c.check_weight_codes()
     c.check_act_codes()
@@ -194,7 +201,8 @@ def test_dynamic_activation_scale(cuda_device):
     assert float(svdq.calibrate_act(c.Xd, c.w).item()) == c.g_x_ref
 
 
-@pytest.mark.parametrize("M,K,N,r,swiglu", [(130, 256, 384, 16, False), (200, 512, 512, 32, True)])
+@pytest.mark.parametrize("M,K,N,r,swiglu", [(130, 256, 384, 16, False), (200, 512, 512, 32, True),
+                                            (130, 256, 768, 16, False)])
 def test_outputs_stay_inside_y(cuda_device, M, K, N, r, swiglu):
     """Canaries: Y is the first M rows of a larger buffer filled with a marker value; after the GEMM
     the rows past M still hold the marker (the output TMA stores clip at row M, although the tile
@@ -214,13 +222,15 @@ def test_outputs_stay_inside_y(cuda_device, M, K, N, r, swiglu):
 
 
 MULTI_TILE = [
-    # more tiles than resident CTA pairs on 192- and 128-wide tiles (the full-size workloads all
-    # use 256-wide ones): the 128-wide kernel's double-buffered accumulators and the barrier phases
-    # carried from tile to tile.      pair tiles = ceil(M / 256) x N / n_tile
+    # more tiles than resident CTA pairs on 384-, 192- and 128-wide tiles (the full-size workloads
+    # use 384- and 256-wide ones): the 128-wide kernel's double-buffered accumulators and the
+    # barrier phases carried from tile to tile.      pair tiles = ceil(M / 256) x N / n_tile
     (2048, 512, 4736, 32, True, False),   # 128-wide: 8 x 37 = 296 tiles
     (1280, 256, 4736, 16, False, True),   # 128-wide SwiGLU: 5 x 37 = 185 tiles
     (1536, 512, 5760, 32, True, False),   # 192-wide: 6 x 30 = 180 tiles
     (1100, 256, 5760, 64, True, True),    # 192-wide SwiGLU, r = 64, ragged last row block: 5 x 30
+    (2048, 512, 9216, 32, True, False),   # 384-wide: 8 x 24 = 192 tiles
+    (1100, 256, 6912, 16, False, False),  # 384-wide, ragged last row block: 5 x 18 = 90 tiles
 ]
 
 

@@ -12,16 +12,16 @@ the issuer waits for full and sf_full, issues the MMAs and commits to both CTAs'
 At the end each producer waits for the release of every slot it filled, so no copy is in flight
 when its CTA exits.
 
-Both accumulator modes are covered: one 256- or 192-column buffer (NVFP4, 5-stage ring), and two
-buffers used alternately (NVFP4 128-wide tiles with a 6-stage ring, and every FP8 tile width with
-6- and 8-stage rings, where without scale factors the issuer waits on the full barrier alone).
+Both accumulator modes are covered: one 256- or 192-column buffer (NVFP4, 5-stage ring, 4 scale
+buffers), one 384-column buffer (NVFP4, 4-stage ring, 2 scale buffers), and two buffers used
+alternately (NVFP4 128-wide tiles with a 6-stage ring, and every FP8 tile width with 6- and 8-stage
+rings, where without scale factors the issuer waits on the full barrier alone).
 Checked: no deadlock, no stray arrival, waits on exactly their completion, no resource used before
 its previous user is done; removing any one wait must make it fail."""
 import random
 
 import pytest
 
-SF_BUFS = 4
 WAITS = ["producer.empty", "producer.drain", "issuer.acce", "issuer.full", "issuer.sf_full", "sf.land",
          "sf.release", "epi.accf"]
 
@@ -38,7 +38,8 @@ class Barrier:
             self.pending = self.count
 
 
-def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=(), scales=True):
+def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=(), scales=True, sf_bufs=4):
+    SF_BUFS = sf_bufs
     rng = random.Random(seed)
     lr_slots = (r + 31) // 32
     slots = lr_slots + k_iters
@@ -198,29 +199,31 @@ def run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip=(), scales=True)
     return True
 
 
-# (stages, accumulator buffers, scale factors) of the kernel's instantiations: NVFP4 256 / 192 ->
-# (5, 1), NVFP4 128 -> (6, 2); row-wise FP8 256 / 192 -> (6, 2, no scales), 128 -> (8, 2, no scales)
-MODES = [(5, 1, True), (6, 2, True), (6, 2, False), (8, 2, False)]
+# (stages, accumulator buffers, scale factors, scale buffers) of the kernel's instantiations:
+# NVFP4 256 / 192 -> (5, 1, 4 buffers), NVFP4 384 -> (4, 1, 2 buffers), NVFP4 128 -> (6, 2, 4
+# buffers); row-wise FP8 256 / 192 -> (6, 2, no scales), 128 -> (8, 2, no scales)
+MODES = [(5, 1, True, 4), (4, 1, True, 2), (6, 2, True, 4), (6, 2, False, 4), (8, 2, False, 4)]
 
 
-@pytest.mark.parametrize("stages,acc_bufs,scales", MODES)
+@pytest.mark.parametrize("stages,acc_bufs,scales,sf_bufs", MODES)
 @pytest.mark.parametrize("n_tiles", [1, 2, 3, 8])
 @pytest.mark.parametrize("r,k_iters", [(32, 1), (64, 2), (0, 3), (16, 12)])
-def test_pair_gemm_protocol_model(stages, acc_bufs, scales, n_tiles, r, k_iters):
+def test_pair_gemm_protocol_model(stages, acc_bufs, scales, sf_bufs, n_tiles, r, k_iters):
     for seed in range(5):
-        assert run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, scales=scales)
+        assert run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, scales=scales, sf_bufs=sf_bufs)
 
 
 @pytest.mark.parametrize("skipped", WAITS)
-@pytest.mark.parametrize("stages,acc_bufs,scales", MODES)
-def test_every_wait_is_needed(skipped, stages, acc_bufs, scales):
+@pytest.mark.parametrize("stages,acc_bufs,scales,sf_bufs", MODES)
+def test_every_wait_is_needed(skipped, stages, acc_bufs, scales, sf_bufs):
     if not scales and skipped.startswith(("sf.", "issuer.sf_")):
         pytest.skip("no scale factors in this format")
     for n_tiles in (3, 8):
         for r, k_iters in ((32, 1), (0, 3), (16, 12)):
             for seed in range(20):
                 try:
-                    run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip={skipped}, scales=scales)
+                    run_model(n_tiles, r, k_iters, stages, acc_bufs, seed, skip={skipped}, scales=scales,
+                              sf_bufs=sf_bufs)
                 except AssertionError:
                     return
     pytest.fail(f"removing the wait {skipped} went unnoticed")
