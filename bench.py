@@ -42,9 +42,9 @@ FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch of the GEMM, from the ncu capture summarised in
 # profiles/pair_gemm_kernel_qkv2048.md, keyed by a hash of the kernel source it was taken on; any
 # change to the kernel source makes the figure stale and it is reported as null.
-PROFILED_GEMM_TRAFFIC = {("qkv_2048", "5b52a0257f1d"): 49.85e6 + 258.10e6}
+PROFILED_GEMM_TRAFFIC = {("qkv_2048", "8e84620ea1f7"): 49.91e6 + 260.21e6}
 # The same for kernel 1 (profiles/quant_act_kernel_qkv2048.md), keyed by a hash of its source.
-PROFILED_K1_TRAFFIC = {("qkv_2048", "bcced91f73dc"): 104.06e6 + 6.44e6}
+PROFILED_K1_TRAFFIC = {("qkv_2048", "827b95adc774"): 104.06e6 + 5.98e6}
 
 
 def read_peaks():
