@@ -537,8 +537,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int e = 0; e < 8; e += 2) {
                 const float z0 = fmaf(alpha, gg[i + e], bg[e]), z1 = fmaf(alpha, gg[i + e + 1], bg[e + 1]);
-                const float y0 = __fdividef(z0, 1.0f + __expf(-z0)) * fmaf(alpha, uu[i + e], bu[e]);
-                const float y1 = __fdividef(z1, 1.0f + __expf(-z1)) * fmaf(alpha, uu[i + e + 1], bu[e + 1]);
+                const float y0 = silu_times(z0, fmaf(alpha, uu[i + e], bu[e]));
+                const float y1 = silu_times(z1, fmaf(alpha, uu[i + e + 1], bu[e + 1]));
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
                 w[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
               }

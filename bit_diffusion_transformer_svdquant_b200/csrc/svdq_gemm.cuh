@@ -695,8 +695,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                   const float z0 = gg[i + e], z1 = gg[i + e + 1];
-                  const float y0 = __fdividef(z0, 1.0f + __expf(-z0)) * uu[i + e];
-                  const float y1 = __fdividef(z1, 1.0f + __expf(-z1)) * uu[i + e + 1];
+                  const float y0 = silu_times(z0, uu[i + e]);
+                  const float y1 = silu_times(z1, uu[i + e + 1]);
                   const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
                   w[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
@@ -724,7 +724,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             affine(ep, up, g0 + kHalf, hN + j0);
             // the same arithmetic as the bf16 path, so that bf16 output = bf16(fp32 output)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) gt[i] = __fdividef(gt[i], 1.0f + __expf(-gt[i])) * up[i];
+            for (int i = 0; i < 32; ++i) gt[i] = silu_times(gt[i], up[i]);
             emit_f32(gt, row0, j0);
           }
         }

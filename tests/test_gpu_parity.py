@@ -140,12 +140,13 @@ def test_full_size_workload(cuda_device, spec):
     c.check_outputs(samples=3000)
 
 
-def test_cuda_graph_replay(cuda_device):
+@pytest.mark.parametrize("N", [512, 768])  # 256- and 384-wide GEMM tiles
+def test_cuda_graph_replay(cuda_device, N):
     """Both kernels captured in a CUDA graph and replayed give the eager result bit for bit (the
     library enqueues everything on the caller's stream and allocates nothing per call), in bf16 and
     fp32 output modes; the replayed activation codes and scales equal the oracle's, and the replayed
     fp32 output is within 2e-3 of max|y_ref| of the oracle's layer."""
-    X, W, b = _rand_layer(300, 768, 512, 32, seed=11, bias=True)
+    X, W, b = _rand_layer(300, 768, N, 32, seed=11, bias=True)
     c = Case(X, W, b, 32, False, cuda_device)
     for dt in (torch.bfloat16, torch.float32):
         y_eager = c.run_gemm(dt).clone()
@@ -174,13 +175,14 @@ def test_cuda_graph_replay(cuda_device):
         del g
 
 
-def test_lora_on_the_branch(cuda_device):
+@pytest.mark.parametrize("N", [512, 768])  # 256- and 384-wide GEMM tiles
+def test_lora_on_the_branch(cuda_device, N):
     """A rank-32 LoRA adapter concatenated onto the rank-32 branch (r = 64 through the same
     kernels) matches the oracle's base layer + X A B."""
-    X, W, b = _rand_layer(300, 768, 512, 32, seed=13, bias=True)
+    X, W, b = _rand_layer(300, 768, N, 32, seed=13, bias=True)
     rng = np.random.default_rng(17)
     A = svdquant.bf16_round(rng.standard_normal((768, 32)) / np.sqrt(768))
-    B = svdquant.bf16_round(rng.standard_normal((32, 512)) * 0.05)
+    B = svdquant.bf16_round(rng.standard_normal((32, N)) * 0.05)
     prep = svdquant.add_lora(svdquant.prepare_layer(X, W, 32), A, B)
     c = Case(X, W, b, 64, False, cuda_device, prep=prep)
     c.check_scales()
