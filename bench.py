@@ -42,9 +42,9 @@ FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch of the GEMM, from the ncu capture summarised in
 # profiles/pair_gemm_kernel_qkv2048.md, keyed by a hash of the kernel source it was taken on; any
 # change to the kernel source makes the figure stale and it is reported as null.
-PROFILED_GEMM_TRAFFIC = {("qkv_2048", "8e84620ea1f7"): 49.91e6 + 260.21e6}
+PROFILED_GEMM_TRAFFIC = {("qkv_2048", "f42f6c5c39d7"): 50.25e6 + 259.95e6}
 # The same for kernel 1 (profiles/quant_act_kernel_qkv2048.md), keyed by a hash of its source.
-PROFILED_K1_TRAFFIC = {("qkv_2048", "827b95adc774"): 104.06e6 + 5.98e6}
+PROFILED_K1_TRAFFIC = {("qkv_2048", "815e7ce8aec3"): 104.06e6 + 5.97e6}
 
 
 def read_peaks():
@@ -664,6 +664,21 @@ def config_row_arm(args, dev):
     ms, parts, _ = two_pass(run, 2 * n_l, K, flush, stream, dev)
     if svdq.device_status() != 0:
         raise RuntimeError("device wait ran out")
+    # the same step captured once in a CUDA graph and replayed, under the same protocol: where the
+    # layer is small, the launches are a visible part of the step
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        run_step(layers)
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_step(layers)
+    graph.replay()
+    graph_ms = time_per_step(graph.replay, K, flush, stream)
+    del graph
+    if svdq.device_status() != 0:
+        raise RuntimeError("device wait ran out in the graph replays")
     k1 = [parts[2 * i] for i in range(n_l)]
     k2 = [parts[2 * i + 1] for i in range(n_l)]
     peaks = read_peaks()
@@ -679,6 +694,7 @@ def config_row_arm(args, dev):
             "gemm_us": [round(x * 1e3, 2) for x in k2],
             "gemm_frac_fp4_peak": [round(gemm_kernel_flops(L["spec"]) / (x * 1e-3) / 1e12 / fp4_peak, 4)
                                    for L, x in zip(layers, k2)],
+            "cuda_graph_ms_per_step": round(graph_ms, 5),
             "steps": K}
 
 
