@@ -328,6 +328,29 @@ def gpu_arm(args, rank, world, dev):
 
     e2e = e2e_arm(args, layers, dev, world)
 
+    # The same steps after a flush that leaves clean lines (the 256 MB write followed by a 256 MB
+    # read): kernel 1, the first kernel of a step, then does not also write back the write-flush's
+    # dirty lines. Reported beside the headline, which keeps the plain write-flush.
+    clean_side = None
+    if clean is None:
+        clean_buf = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        c_ms, c_parts, _ = two_pass(run, per * n_l, min(K, 50), flush, stream, dev, clean_buf)
+        del clean_buf
+        c_k1 = [c_parts[per * i + per - 2] for i in range(n_l)]
+        c_k2 = [c_parts[per * i + per - 1] for i in range(n_l)]
+        c_ms = max_over_ranks(c_ms, dev)
+        clean_side = {
+            "ms_per_step": round(c_ms, 5),
+            "frac_fp4_peak_e2e": round(flops_main / (c_ms * 1e-3) / 1e12 / fp4_peak, 4),
+            "quantize_act_us": [round(x * 1e3, 2) for x in c_k1],
+            "quantize_act_frac_hbm": [round(kernel1_bytes(layers[i]["spec"]) / (c_k1[i] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+                                      for i in range(n_l)],
+            "gemm_us": [round(x * 1e3, 2) for x in c_k2],
+            "what": "the same steps with a 256 MB read after each 256 MB write-flush (outside the events), so "
+                    "that each step starts on clean L2 lines"}
+        if svdq.device_status() != 0:
+            raise RuntimeError("device wait ran out in the clean-flush pass")
+
     # The same step replayed from a CUDA graph (both kernels of every layer captured once), and the
     # bf16 cuBLAS baseline on the same shapes; same timing protocol, fewer steps.
     side_steps = max(3, min(K, 50))
@@ -401,6 +424,7 @@ def gpu_arm(args, rank, world, dev):
         "gpu_launches": (4 if dyn else 2) * n_l * K,
         "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 3),
+        **({"l2_clean_variant": clean_side} if clean_side is not None else {}),
     }
     return out
 
