@@ -18,15 +18,15 @@
 //                of L2^T in chunks of 32 columns of r.
 //   warp 1       TMEM allocation for the pair; in the even CTA also the MMA issuer: per ring slot
 //                it waits for the slot's barrier in the even CTA (8 arrivals: the scale writers of
-//                both CTAs), issues 4 x tcgen05.mma kind::mxf4nvf4 (M=256, N=n_tile, K=64) or the
-//                low-rank kind::f16 MMAs, and multicasts one commit to the slot's empty barrier in
-//                both CTAs.
+//                both CTAs), issues 4 x tcgen05.mma kind::mxf4nvf4 (M=256, N=n_tile, K=64; at
+//                n_tile 384 each as N=256 + N=128) or the low-rank kind::f16 MMAs, and multicasts
+//                one commit to the slot's empty barrier in both CTAs.
 //   warps 2..9   epilogue: two warps per 32-lane TMEM quadrant, each half of the tile's columns:
 //                tcgen05.ld, y = alpha acc (+ bias), SwiGLU on interleaved gate/up columns, into a
 //                swizzled staging buffer, TMA store. The accumulator goes back to the issuer (a
 //                remote arrive) as soon as its last columns are in registers.
 //   warps 10..13 scale-factor writers: per ring slot, wait for this CTA's data, copy the scale
-//                atoms from shared memory into one of 4 TMEM scale buffers with tcgen05.st (each
+//                atoms from shared memory into one of the TMEM scale buffers with tcgen05.st (each
 //                warp its lane quadrant), then arrive on the issuer's barrier in the even CTA.
 //                Measured on B200, every tcgen05.cp costs ~64 tensor-pipe cycles whatever its
 //                shape, so copying 12 atoms per K step with tcgen05.cp starved the MMAs; stores
