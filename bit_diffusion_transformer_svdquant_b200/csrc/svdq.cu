@@ -1184,7 +1184,7 @@ svdq_status svdq_fp8r_export_act(const svdq_fp8r_act* act, uint8_t* codes, float
 namespace {
 
 constexpr int kFusedStages = 5;
-constexpr int kMaxSplits = 8;
+constexpr int kMaxSplits = svdq::fused::kMaxUSplits;
 
 struct FusedState {
   bool ready = false;

@@ -622,9 +622,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// The most column splits a unit schedule uses (the partials buffer holds this many slices).
+constexpr int kMaxUSplits = 8;
+
 // U' = sum over splits of the partial sums (in split order), stored as kernel 1 stores U: u =
 // fp32(U' * fp32(1 / alpha')) with alpha' = fp32(g_x' g_w'), as bf16 hi = bf16(u) and lo =
-// bf16(u - hi); rows past M are zero. Also writes alpha'.
+// bf16(u - hi); rows past M are zero. Also writes alpha'. A thread issues all its partial loads
+// before the first sum, so their latencies overlap.
 __global__ void finalize_u_kernel(const float* __restrict__ partials, int splits, int M, int M_pad, int r,
                                   const float* g_x2, const float* g_w2, __nv_bfloat16* __restrict__ U,
                                   float* alpha_out) {
@@ -637,9 +641,14 @@ __global__ void finalize_u_kernel(const float* __restrict__ partials, int splits
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int m = static_cast<int>(i / r);
+    float pv[kMaxUSplits];
+#pragma unroll
+    for (int sp = 0; sp < kMaxUSplits; ++sp)
+      pv[sp] = (m < M && sp < splits) ? partials[static_cast<size_t>(sp) * total + i] : 0.0f;
     float s = 0.0f;
-    if (m < M)
-      for (int sp = 0; sp < splits; ++sp) s += partials[static_cast<size_t>(sp) * total + i];
+#pragma unroll
+    for (int sp = 0; sp < kMaxUSplits; ++sp)
+      if (sp < splits) s += pv[sp];
     const float v = __fmul_rn(s, cinv);
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     U[i] = hi;

@@ -145,9 +145,10 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr) : "memory");
   return v;
 }
 
@@ -202,7 +203,9 @@ struct Q1Layout {
   static constexpr int kLamOff = kQTile + kL1;      // the stage's 64 inverse smoothing factors (fp32)
   static constexpr int kStage = kQTile + kL1 + 1024;
   static constexpr int kPartOff = kStages * kStage;
-  static constexpr int kPart = R * 128 * 4 + 128 * 4;  // rows padded to R + 1 floats
+  // a cluster member's partial U: 128 rows padded to R + 4 floats (16-byte rows, conflict-free
+  // 16-byte accesses per quarter warp)
+  static constexpr int kPart = (R + 4) * 128 * 4;
   static constexpr int kTabOff = kPartOff + kPart;        // 128 fp32: 1 / (dec(s) g_x) per scale code
   static constexpr int kBarOff = kTabOff + 128 * 4;
   static constexpr int kNumBars = 2 * kStages + 2;
@@ -505,18 +508,33 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
           }
         }
         if (csize > 1 && crank != 0) {
-          float* part = reinterpret_cast<float*>(smem + L::kPartOff) + (q * 32 + lane) * (R + 1);
+          float4* part = reinterpret_cast<float4*>(smem + L::kPartOff) + (q * 32 + lane) * ((R + 4) / 4);
 #pragma unroll
-          for (int j = 0; j < R; ++j) part[j] = u[j];
+          for (int j = 0; j < R; j += 4) part[j / 4] = make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
         }
       }
       if (csize > 1) cluster_sync_all();
       if (got && crank == 0) {
         const int rl = q * 32 + lane;
+        // 16-byte remote loads, kInFlight of them before their sums (fewer at r = 64, whose 64
+        // values per row already take most registers): with one 4-byte load per value, the two
+        // peers' 64 loads per row took ~7 us on B200
+        constexpr int kInFlight = R >= 64 ? 2 : 4;
         for (uint32_t rk = 1; rk < csize; ++rk) {
-          const uint32_t pa = cluster_map(smem_addr(smem + L::kPartOff) + rl * (R + 1) * 4, rk);
+          const uint32_t pa = cluster_map(smem_addr(smem + L::kPartOff) + rl * (R + 4) * 4, rk);
 #pragma unroll
-          for (int j = 0; j < R; ++j) u[j] += ld_cluster_f32(pa + j * 4);
+          for (int j0 = 0; j0 < R; j0 += 4 * kInFlight) {
+            float4 pv[kInFlight];
+#pragma unroll
+            for (int e = 0; e < kInFlight; ++e) pv[e] = ld_cluster_v4(pa + (j0 + 4 * e) * 4);
+#pragma unroll
+            for (int e = 0; e < kInFlight; ++e) {
+              u[j0 + 4 * e] += pv[e].x;
+              u[j0 + 4 * e + 1] += pv[e].y;
+              u[j0 + 4 * e + 2] += pv[e].z;
+              u[j0 + 4 * e + 3] += pv[e].w;
+            }
+          }
         }
         const float cinv = Q::u_scale(a, m_tile * 128 + rl);
         __nv_bfloat16* u_hi = a.U + (static_cast<size_t>(m_tile) * 128 + rl) * R;
