@@ -516,10 +516,11 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       if (csize > 1) cluster_sync_all();
       if (got && crank == 0) {
         const int rl = q * 32 + lane;
-        // 16-byte remote loads, kInFlight of them before their sums (fewer at r = 64, whose 64
-        // values per row already take most registers): with one 4-byte load per value, the two
-        // peers' 64 loads per row took ~7 us on B200
-        constexpr int kInFlight = R >= 64 ? 2 : 4;
+        // 16-byte remote loads, a peer's whole row (2 at a time at r = 64, whose 64 values per row
+        // already take most registers) in flight before the sums: with one 4-byte load per value,
+        // the two peers' 64 loads per row took ~7 us on B200
+        constexpr int kInFlight = R >= 64 ? 2 : (R / 4 < 8 ? R / 4 : 8);
+        static_assert(R % (4 * kInFlight) == 0, "whole batches of 16-byte loads per row");
         for (uint32_t rk = 1; rk < csize; ++rk) {
           const uint32_t pa = cluster_map(smem_addr(smem + L::kPartOff) + rl * (R + 4) * 4, rk);
 #pragma unroll
