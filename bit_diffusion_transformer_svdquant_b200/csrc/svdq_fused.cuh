@@ -436,6 +436,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const float alpha = *args.alpha;
     const float gx2 = *args.g_x2;
     const float d6 = __fmul_rn(6.0f, gx2);
+    const float rd6 = __frcp_rn(d6);
     const float* rs_tab = reinterpret_cast<const float*>(smem + L::kTabOff);
     const bool has_bias = args.bias != nullptr;
     const int hN = args.N >> 1;
@@ -585,13 +586,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             }
 #pragma unroll
             for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
-            uint32_t sc = row < args.M ? cvt_e4m3(__fdiv_rn(amax, d6)) : 0u;
+            // kernel 1's scale rule: the reciprocal multiply, with the exact division only near an
+            // E4M3 rounding boundary or below E4M3's normal range (the same code either way)
+            float qs = __fmul_rn(amax, rd6);
+            if (scale_needs_division(qs)) qs = __fdiv_rn(amax, d6);
+            uint32_t sc = row < args.M ? cvt_e4m3(qs) : 0u;
             uint2 codes = make_uint2(0u, 0u);
             if (sc != 0) {
               const float rr = rs_tab[sc];
+              const float2 r2 = make_float2(rr, rr);
               float qv[16];
 #pragma unroll
-              for (int e = 0; e < 16; ++e) qv[e] = __fmul_rn(v[e], rr);
+              for (int e = 0; e < 16; e += 2) {
+                const float2 p = mul2_rn(make_float2(v[e], v[e + 1]), r2);
+                qv[e] = p.x;
+                qv[e + 1] = p.y;
+              }
               codes.x = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(qv));
               codes.y = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(qv + 8));
             }

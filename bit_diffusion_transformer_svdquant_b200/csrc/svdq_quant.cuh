@@ -182,7 +182,7 @@ __device__ __forceinline__ bool scale_needs_division(float q) {
 // RowAct in svdq_fp8r.cuh) and the scale U is stored with.
 //
 // A CTA (one per SM) owns 128 rows of X and a K range: the whole K, or a share of it when a
-// thread-block cluster of 2 or 4 CTAs splits K so that few row tiles still fill the SMs in one
+// thread-block cluster of 2, 3 or 4 CTAs splits K so that few row tiles still fill the SMs in one
 // wave. TMA streams 128 x 64 bf16 stages (128B swizzle; an L2 evict-first policy, since X is read
 // once) of X, the stage's 64-column slice of L1s^T and its 64 inverse smoothing factors into an
 // 8-deep shared-memory ring (6 at r = 64). Every stage is read twice from shared memory: by one of
