@@ -145,11 +145,13 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr) : "memory");
-  return v;
+// Generic address of the same shared-memory location in CTA `rank` of the cluster (plain loads
+// through it read that CTA's shared memory).
+template <class T>
+__device__ __forceinline__ const T* cluster_map_generic(const T* p, uint32_t rank) {
+  uint64_t r;
+  asm volatile("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+  return reinterpret_cast<const T*>(r);
 }
 
 // Largest magnitude of 16 values, as a balanced tree of 3-input maxima (depth 3 instead of a
@@ -516,24 +518,33 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       if (csize > 1) cluster_sync_all();
       if (got && crank == 0) {
         const int rl = q * 32 + lane;
-        // 16-byte remote loads, a peer's whole row (2 at a time at r = 64, whose 64 values per row
-        // already take most registers) in flight before the sums: with one 4-byte load per value,
-        // the two peers' 64 loads per row took ~7 us on B200
-        constexpr int kInFlight = R >= 64 ? 2 : (R / 4 < 8 ? R / 4 : 8);
-        static_assert(R % (4 * kInFlight) == 0, "whole batches of 16-byte loads per row");
+        // A peer's whole row of loads in flight before the sums, 16 bytes each up to r = 32: with
+        // one 4-byte load per value at a time, the two peers' 64 loads per row took ~7 us on B200.
+        // At r = 64, whose 64 values per row already take most registers, 4-byte loads 16 at a time
+        // (16-byte loads there cost the main loop spills).
         for (uint32_t rk = 1; rk < csize; ++rk) {
-          const uint32_t pa = cluster_map(smem_addr(smem + L::kPartOff) + rl * (R + 4) * 4, rk);
+          if constexpr (R <= 32) {
+            const float4* pg =
+                cluster_map_generic(reinterpret_cast<const float4*>(smem + L::kPartOff) + rl * ((R + 4) / 4), rk);
+            float4 pv[R / 4];
 #pragma unroll
-          for (int j0 = 0; j0 < R; j0 += 4 * kInFlight) {
-            float4 pv[kInFlight];
+            for (int e = 0; e < R / 4; ++e) pv[e] = pg[e];
 #pragma unroll
-            for (int e = 0; e < kInFlight; ++e) pv[e] = ld_cluster_v4(pa + (j0 + 4 * e) * 4);
+            for (int e = 0; e < R / 4; ++e) {
+              u[4 * e] += pv[e].x;
+              u[4 * e + 1] += pv[e].y;
+              u[4 * e + 2] += pv[e].z;
+              u[4 * e + 3] += pv[e].w;
+            }
+          } else {
+            const float* pg = cluster_map_generic(reinterpret_cast<const float*>(smem + L::kPartOff) + rl * (R + 4), rk);
 #pragma unroll
-            for (int e = 0; e < kInFlight; ++e) {
-              u[j0 + 4 * e] += pv[e].x;
-              u[j0 + 4 * e + 1] += pv[e].y;
-              u[j0 + 4 * e + 2] += pv[e].z;
-              u[j0 + 4 * e + 3] += pv[e].w;
+            for (int j0 = 0; j0 < R; j0 += 16) {
+              float pv[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pv[e] = pg[j0 + e];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) u[j0 + e] += pv[e];
             }
           }
         }
