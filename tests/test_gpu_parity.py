@@ -297,3 +297,27 @@ def test_weight_bind_offsets_match_pack(cuda_device):
     for f in _DESC_PTRS:
         assert getattr(d, f) - blob.data_ptr() == getattr(c.w.desc, f) - c.w.buf.data_ptr(), f
     assert (d.N, d.K, d.r, d.n_tile, d.swiglu_interleaved) == (c.w.N, c.w.K, c.w.r, c.w.n_tile, 0)
+
+
+@pytest.mark.parametrize("r", [16, 32, 64])
+@pytest.mark.parametrize("cluster", ["1", "2", "3", "4"])
+def test_kernel1_cluster_sizes(cuda_device, monkeypatch, cluster, r):
+    """Kernel 1 with K split over thread-block clusters of 1 to 4 CTAs (SVDQ_K1_CLUSTER), at every
+    branch rank: the leader's sum of its peers' partial U (16-byte loads up to r = 32, 4-byte loads
+    at r = 64) must keep codes and scales bit-exact and the outputs within 2e-3 of the oracle, and
+    U must not depend on the split (the sums run in rank order; rounding aside, the same values)."""
+    X, W, b = _rand_layer(300, 768, 512, r, seed=77 + r, bias=True)
+    monkeypatch.setenv("SVDQ_K1_CLUSTER", cluster)
+    c = Case(X, W, b, r, False, cuda_device)
+    c.check_scales()
+    c.check_act_codes()
+    c.check_outputs()
+    u_split = c.act.U().float().clone()
+    monkeypatch.setenv("SVDQ_K1_CLUSTER", "1")
+    svdq.quantize_act(c.Xd, c.w, c.g_x, c.act)
+    torch.cuda.synchronize(cuda_device)
+    assert svdq.device_status() == 0
+    u_one = c.act.U().float()
+    # hi + lo of U: fp32 partial sums in another order differ by rounding only
+    tot_split, tot_one = u_split[0] + u_split[1], u_one[0] + u_one[1]
+    assert float((tot_split - tot_one).abs().max()) <= 1e-4 * float(tot_one.abs().max()) + 1e-30
