@@ -148,10 +148,10 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
 // Generic address of the same shared-memory location in CTA `rank` of the cluster (plain loads
 // through it read that CTA's shared memory).
 template <class T>
-__device__ __forceinline__ const T* cluster_map_generic(const T* p, uint32_t rank) {
+__device__ __forceinline__ T* cluster_map_generic(T* p, uint32_t rank) {
   uint64_t r;
   asm volatile("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
-  return reinterpret_cast<const T*>(r);
+  return reinterpret_cast<T*>(r);
 }
 
 // Largest magnitude of 16 values, as a balanced tree of 3-input maxima (depth 3 instead of a
@@ -206,9 +206,11 @@ struct Q1Layout {
   static constexpr int kStage = kQTile + kL1 + 1024;
   static constexpr int kPartOff = kStages * kStage;
   // a cluster member's partial U: 128 rows padded to R + 4 floats (16-byte rows, conflict-free
-  // 16-byte accesses per quarter warp)
+  // 16-byte accesses per quarter warp). Up to r = 32 the leader holds one slot per peer (at most 3),
+  // which the peers write into; at r = 64 each CTA keeps its own, which the leader reads.
   static constexpr int kPart = (R + 4) * 128 * 4;
-  static constexpr int kTabOff = kPartOff + kPart;        // 128 fp32: 1 / (dec(s) g_x) per scale code
+  static constexpr int kPartSlots = R <= 32 ? 3 : 1;
+  static constexpr int kTabOff = kPartOff + kPartSlots * kPart;  // 128 fp32: 1 / (dec(s) g_x) per scale code
   static constexpr int kBarOff = kTabOff + 128 * 4;
   static constexpr int kNumBars = 2 * kStages + 2;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;
@@ -510,7 +512,11 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
           }
         }
         if (csize > 1 && crank != 0) {
-          float4* part = reinterpret_cast<float4*>(smem + L::kPartOff) + (q * 32 + lane) * ((R + 4) / 4);
+          // up to r = 32 straight into the leader's slot for this rank (remote stores do not wait
+          // for a reply; the cluster barrier below makes them visible), at r = 64 into this CTA
+          float4* part = reinterpret_cast<float4*>(smem + L::kPartOff + (R <= 32 ? (crank - 1) * L::kPart : 0)) +
+                         (q * 32 + lane) * ((R + 4) / 4);
+          if constexpr (R <= 32) part = cluster_map_generic(part, 0);
 #pragma unroll
           for (int j = 0; j < R; j += 4) part[j / 4] = make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
         }
@@ -518,14 +524,13 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       if (csize > 1) cluster_sync_all();
       if (got && crank == 0) {
         const int rl = q * 32 + lane;
-        // A peer's whole row of loads in flight before the sums, 16 bytes each up to r = 32: with
-        // one 4-byte load per value at a time, the two peers' 64 loads per row took ~7 us on B200.
-        // At r = 64, whose 64 values per row already take most registers, 4-byte loads 16 at a time
-        // (16-byte loads there cost the main loop spills).
+        // Up to r = 32 the peers' rows are already in this CTA's slots. At r = 64, whose 64 values per
+        // row already take most registers, the leader reads each peer's row with 4-byte remote loads,
+        // 16 at a time. (One 4-byte remote load per value at a time took ~7 us on B200 for two peers.)
         for (uint32_t rk = 1; rk < csize; ++rk) {
           if constexpr (R <= 32) {
             const float4* pg =
-                cluster_map_generic(reinterpret_cast<const float4*>(smem + L::kPartOff) + rl * ((R + 4) / 4), rk);
+                reinterpret_cast<const float4*>(smem + L::kPartOff + (rk - 1) * L::kPart) + rl * ((R + 4) / 4);
             float4 pv[R / 4];
 #pragma unroll
             for (int e = 0; e < R / 4; ++e) pv[e] = pg[e];
